@@ -1,0 +1,186 @@
+"""ctypes binding of libra.so (argument marshalling only).
+
+Every call forwards torch tensors' device pointers and sizes to the C ABI declared in
+include/ra.h and launches on torch's current CUDA stream. PyTorch provides device memory
+and streams; all arithmetic of the path runs in the library's CUDA kernels. There is no
+CPU fallback: a missing library raises on first use.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+library_path = os.environ.get("RA_LIBRARY", os.path.join(_PKG, "libra.so"))
+
+RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_CUDA, RA_ERR_TIMEOUT, RA_ERR_DEVICE_BOUNDS = range(6)
+RA_F32, RA_BF16 = 0, 1
+LAYOUTS = {"contiguous": 0, "striped": 1, "zigzag": 2}
+
+# name -> (restype, argtypes) of every symbol include/ra.h declares
+_i64, _i32, _f32, _vp = ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_void_p
+SIGNATURES = {
+    "ra_partial": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i64, _i64, _i32, _f32, _i32,
+                          _i64, _i64, _i64, _i64, _vp, _vp, _vp]),
+    "ra_merge": (_i32, [_vp, _vp, _i32, _i64, _i32, _vp, _i32, _vp, _vp]),
+    "ra_ring_forward": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i64, _i32, _f32, _i32, _i32,
+                               _i32, _vp, _vp, _vp]),
+    "ra_status_string": (ctypes.c_char_p, [_i32]),
+    "ra_get_device_error": (_i32, [_vp]),
+    "ra_abi_version": (_i32, []),
+}
+
+_lock = threading.Lock()
+_handle = None
+
+
+class RaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+def load():
+    """Load libra.so once and declare the C signatures. Raises if the library is missing."""
+    global _handle
+    with _lock:
+        if _handle is None:
+            if not os.path.exists(library_path):
+                raise RuntimeError(
+                    f"libra.so not found at {library_path}: build it with "
+                    "`python -m sequence_softmax_b200.build` (there is no CPU fallback)")
+            lib = ctypes.CDLL(library_path)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _handle = lib
+    return _handle
+
+
+def status_string(status: int) -> str:
+    return load().ra_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != RA_OK:
+        raise RaError(status, what)
+
+
+def _stream_ptr(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return RA_F32
+    if t.dtype == torch.bfloat16:
+        return RA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _dev(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def get_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error status code."""
+    return load().ra_get_device_error(_stream_ptr(stream))
+
+
+def partial(q, k, v, causal: bool = False, scale: float | None = None,
+            q_tok0: int = 0, q_tok_stride: int = 1, k_tok0: int = 0, k_tok_stride: int = 1,
+            out=None, lse=None, stream=None):
+    """One query block against one KV chunk -> (O_partial fp32 [B,H,Lq,d], lse fp32 [B,H,Lq])."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    if k.shape != (B, H, Lk, d) or v.shape != k.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("k and v must be [B, H, Lk, d] with q's B, H, d and dtype")
+    scale = d ** -0.5 if scale is None else float(scale)
+    out = torch.empty(B, H, Lq, d, device=q.device, dtype=torch.float32) if out is None else out
+    lse = torch.empty(B, H, Lq, device=q.device, dtype=torch.float32) if lse is None else lse
+    _dev(out, "out")
+    _dev(lse, "lse")
+    st = load().ra_partial(q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q), B, H, Lq, Lk, d, scale,
+                           int(bool(causal)), q_tok0, q_tok_stride, k_tok0, k_tok_stride,
+                           out.data_ptr(), lse.data_ptr(), _stream_ptr(stream))
+    _check(st, "ra_partial")
+    return out, lse
+
+
+def merge(o_parts, lse_parts, out_dtype=torch.bfloat16, with_lse: bool = True, out=None, lse=None,
+          stream=None):
+    """lse-weighted combination of n partial states.
+
+    o_parts [n, ..., d] fp32, lse_parts [n, ...] fp32 -> (O [..., d] out_dtype, L [...] fp32 or None).
+    """
+    _dev(o_parts, "o_parts")
+    _dev(lse_parts, "lse_parts")
+    if o_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32:
+        raise TypeError("partial states are float32")
+    n, d = o_parts.shape[0], o_parts.shape[-1]
+    lead = tuple(o_parts.shape[1:-1])
+    if tuple(lse_parts.shape) != (n, *lead):
+        raise ValueError("lse_parts must be [n, ...] matching o_parts [n, ..., d]")
+    rows = 1
+    for x in lead:
+        rows *= x
+    out = torch.empty(*lead, d, device=o_parts.device, dtype=out_dtype) if out is None else out
+    if with_lse and lse is None:
+        lse = torch.empty(*lead, device=o_parts.device, dtype=torch.float32)
+    _dev(out, "out")
+    st = load().ra_merge(o_parts.data_ptr(), lse_parts.data_ptr(), n, rows, d, out.data_ptr(),
+                         _dtype_code(out), lse.data_ptr() if with_lse else None, _stream_ptr(stream))
+    _check(st, "ra_merge")
+    return out, (lse if with_lse else None)
+
+
+def ring_forward(q, k, v, n_chunks: int, causal: bool = False, layout: str = "contiguous",
+                 scale: float | None = None, return_lse: bool = True, out=None, lse=None, stream=None):
+    """Exact attention by the ordered ring over ``n_chunks`` virtual positions.
+
+    q, k, v [B, H, N, d] (bf16 with d in {64, 128}, or fp32 with d <= 128), natural token order.
+    Returns (O [B,H,N,d] in q's dtype, lse [B,H,N] fp32 or None). Host (CPU) tensors are
+    accepted: they are copied to the current device, the call runs there, and the results
+    are copied back to host memory before returning.
+    """
+    if not q.is_cuda:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        qd, kd, vd = (t.to(dev, non_blocking=True) for t in (q, k, v))
+        o_d, l_d = ring_forward(qd, kd, vd, n_chunks, causal, layout, scale, return_lse, stream=stream)
+        pin = q.is_pinned()
+        o_h = torch.empty(o_d.shape, dtype=o_d.dtype, pin_memory=pin) if out is None else out
+        o_h.copy_(o_d, non_blocking=pin)
+        l_h = None
+        if return_lse:
+            l_h = torch.empty(l_d.shape, dtype=l_d.dtype, pin_memory=pin) if lse is None else lse
+            l_h.copy_(l_d, non_blocking=pin)
+        torch.cuda.current_stream().synchronize()
+        return o_h, l_h
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev(t, n)
+    B, H, N, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share shape [B, H, N, d] and dtype")
+    if layout not in LAYOUTS:
+        raise ValueError(f"layout must be one of {sorted(LAYOUTS)}")
+    scale = d ** -0.5 if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    if return_lse and lse is None:
+        lse = torch.empty(B, H, N, device=q.device, dtype=torch.float32)
+    _dev(out, "out")
+    st = load().ra_ring_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q), B, H, N, d, scale,
+                                int(n_chunks), int(bool(causal)), LAYOUTS[layout], out.data_ptr(),
+                                lse.data_ptr() if return_lse else None, _stream_ptr(stream))
+    _check(st, "ra_ring_forward")
+    return out, (lse if return_lse else None)

@@ -1,0 +1,442 @@
+// attn_tc.cuh -- bf16 ring-attention forward on the 5th-generation tensor cores (sm_100a).
+//
+// One CTA owns a query block of two 128-row tiles of one virtual ring position and walks
+// that position's KV tiles in ring order ([BLOG] ring_attention_forward: position p visits
+// position (p - s) mod P at step s; [GLOSSARY] "How Ring Attention works"), folding each
+// 128-key tile into a running online-softmax state (m, l, o) ([BLOG] blockwise_attention;
+// [CARD] online softmax). Causal tiles wholly in the future are never visited; tiles that
+// straddle the diagonal are masked elementwise ([BLOG] ring_attention_causal_step).
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax for query tile 0 (thread i owns row i = TMEM lane i)
+//   warps 4-7  softmax for query tile 1
+//   warp  8    TMA producer: Q tiles once, then K/V tiles into an NSTAGE ring of shared
+//              memory stages (the single-GPU counterpart of the ring's overlap of the next
+//              chunk's transfer with the current chunk's compute)
+//   warp  9    MMA issuer (one thread): S_t = Q_t K^T (both operands from 128B-swizzled
+//              shared memory) and O_t += P_t V (P from tensor memory, V from shared memory)
+//
+// Tensor memory (512 columns x 128 lanes of fp32): S_0 | S_1 | O_0 | O_1. P_t (bf16 pairs)
+// overwrites the first 64 columns of S_t. The MMA warp issues, per KV tile n,
+//   PV_0(n-1), S_0(n), PV_1(n-1), S_1(n)
+// so the tensor core computes one tile's GEMMs while the other tile's softmax runs. MMAs
+// issued by one thread execute in order, so S_t(n) cannot overwrite P_t(n-1) before
+// PV_t(n-1) has read it, and the commit that signals S_t(n) also covers PV_t(n-1): when a
+// softmax warpgroup sees S_t(n), its O_t is stable and may be rescaled.
+//
+// Rescaling is conditional: the running max used for exponentials only moves when the
+// true row max exceeds it by more than RESCALE_LOG2 (in log2 units); until then exp2 values
+// stay <= 2^RESCALE_LOG2 and l and O keep sharing the same stale max, so the result is
+// exact up to rounding.
+#pragma once
+
+#include "common.cuh"
+
+namespace ra {
+
+constexpr int TC_BM = 128;          // query rows per tile
+constexpr int TC_BN = 128;          // keys per KV tile
+constexpr int TC_THREADS = 320;
+constexpr int TC_WARP_PRODUCER = 8;
+constexpr int TC_WARP_MMA = 9;
+constexpr int TC_TMEM_COLS = 512;
+constexpr float RESCALE_LOG2 = 8.0f;
+
+template <int D>
+struct TcCfg {
+  static_assert(D == 64 || D == 128, "head dimension 64 or 128");
+  static constexpr int BOX_BYTES = TC_BM * 64 * 2;         // one TMA box: 128 rows x 64 bf16
+  static constexpr int NBOX = D / 64;                      // boxes per tile (d split in 64s)
+  static constexpr int TILE_BYTES = NBOX * BOX_BYTES;      // one Q, K or V tile
+  static constexpr int NSTAGE = (D == 128) ? 4 : 8;        // K/V ring depth (in tiles)
+  static constexpr int Q_OFF = 0;
+  static constexpr int KV_OFF = 2 * TILE_BYTES;
+  static constexpr int BAR_OFF = KV_OFF + NSTAGE * TILE_BYTES;
+  static constexpr int NBAR = 2 + 2 * NSTAGE + 2 + 2 + 2 + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack to align the base to 1 KB
+  static constexpr int COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(TC_BM, TC_BN, false);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(TC_BM, D, true);
+};
+
+// Query block owned by CTA `unit` of a head, heaviest (latest tokens) first.
+struct QBlock {
+  int p;      // virtual position
+  Seg seg;    // the position's segment that holds the block
+  int64_t i0; // local row of tile 0 inside the segment
+};
+
+__device__ __forceinline__ QBlock decode_unit(const Plan& pl, int unit) {
+  QBlock b;
+  const int P = pl.P;
+  const int64_t nb = (pl.q_seg_len + 2 * TC_BM - 1) / (2 * TC_BM);
+  int si = 0;
+  int64_t qb;
+  if (pl.layout == RA_LAYOUT_STRIPED) {
+    qb = nb - 1 - unit / P;
+    b.p = P - 1 - unit % P;
+  } else if (pl.layout == RA_LAYOUT_ZIGZAG) {
+    const int gc = 2 * P - 1 - (int)(unit / nb);  // global chunk, latest first
+    qb = nb - 1 - unit % nb;
+    if (gc >= P) { b.p = 2 * P - 1 - gc; si = 1; } else { b.p = gc; si = 0; }
+  } else {
+    b.p = P - 1 - (int)(unit / nb);
+    qb = nb - 1 - unit % nb;
+  }
+  b.seg = segment_of(pl.layout, P, pl.q_seg_len, b.p, si);
+  b.i0 = qb * (2 * TC_BM);
+  return b;
+}
+
+__device__ __forceinline__ int64_t q_token(const Plan& pl, const Seg& s, int64_t i) {
+  return pl.q_tok0 + pl.q_tok_stride * (s.row0 + s.stride * i);
+}
+
+template <int D>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const Plan pl) {
+  using C = TcCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + C::Q_OFF;
+  const uint32_t sKV = sbase + C::KV_OFF;
+  const uint32_t bar0 = sbase + C::BAR_OFF;
+  auto bar_q_full = [&](int t) { return bar0 + 8u * t; };
+  auto bar_kv_full = [&](int s) { return bar0 + 8u * (2 + s); };
+  auto bar_kv_empty = [&](int s) { return bar0 + 8u * (2 + C::NSTAGE + s); };
+  auto bar_s_full = [&](int t) { return bar0 + 8u * (2 + 2 * C::NSTAGE + t); };
+  auto bar_p_full = [&](int t) { return bar0 + 8u * (4 + 2 * C::NSTAGE + t); };
+  auto bar_o_done = [&](int t) { return bar0 + 8u * (6 + 2 * C::NSTAGE + t); };
+  const uint32_t bar_drain = bar0 + 8u * (8 + 2 * C::NSTAGE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x % pl.BH;
+  const int unit = blockIdx.x / pl.BH;
+  const QBlock qb = decode_unit(pl, unit);
+  const int64_t q_last = min(qb.i0 + 2 * TC_BM, qb.seg.count) - 1;  // last valid local row
+  const int64_t tq_max = q_token(pl, qb.seg, q_last);
+  const int nks = num_segments(pl.layout);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q_full(0), 1);
+    mbar_init(bar_q_full(1), 1);
+    for (int s = 0; s < C::NSTAGE; ++s) {
+      mbar_init(bar_kv_full(s), 1);
+      mbar_init(bar_kv_empty(s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar_s_full(t), 1);
+      mbar_init(bar_p_full(t), TC_BM);
+      mbar_init(bar_o_done(t), 1);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == TC_WARP_MMA) {
+    tmem_alloc(smem_u32(tmem_slot), TC_TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == TC_WARP_PRODUCER && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  // Number of KV tiles this block visits (identical walk in every role).
+  int T = 0;
+  for (int s = 0; s < pl.P; ++s) {
+    int c = qb.p - s;
+    if (c < 0) c += pl.P;
+    for (int sk = 0; sk < nks; ++sk) {
+      const Seg ks = segment_of(pl.layout, pl.P, pl.k_seg_len, c, sk);
+      T += (int)((visible_prefix(pl, ks, tq_max) + TC_BN - 1) / TC_BN);
+    }
+  }
+
+  if (warp == TC_WARP_PRODUCER) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const int qy = (int)(qb.seg.row0 % qb.seg.stride);
+      const int64_t qz0 = qb.seg.row0 / qb.seg.stride + qb.i0;
+      for (int t = 0; t < 2; ++t) {
+        mbar_arrive_expect_tx(bar_q_full(t), C::TILE_BYTES);
+        for (int b = 0; b < C::NBOX; ++b)
+          tma_load_4d(sQ + t * C::TILE_BYTES + b * C::BOX_BYTES, &tm_q, bar_q_full(t), 64 * b, qy,
+                      (int)(qz0 + t * TC_BM), bh);
+      }
+      uint32_t use = 0;
+      bool ok = true;
+      for (int s = 0; s < pl.P && ok; ++s) {
+        int c = qb.p - s;
+        if (c < 0) c += pl.P;
+        for (int sk = 0; sk < nks && ok; ++sk) {
+          const Seg ks = segment_of(pl.layout, pl.P, pl.k_seg_len, c, sk);
+          const int ntiles = (int)((visible_prefix(pl, ks, tq_max) + TC_BN - 1) / TC_BN);
+          const int ky = (int)(ks.row0 % ks.stride);
+          const int64_t kz0 = ks.row0 / ks.stride;
+          for (int jt = 0; jt < ntiles && ok; ++jt) {
+            for (int kv = 0; kv < 2; ++kv, ++use) {
+              const int st = use % C::NSTAGE;
+              const uint32_t ph = (use / C::NSTAGE) & 1u;
+              if (!mbar_wait(bar_kv_empty(st), ph ^ 1u, abort_flag)) { ok = false; break; }
+              mbar_arrive_expect_tx(bar_kv_full(st), C::TILE_BYTES);
+              const CUtensorMap* map = kv == 0 ? &tm_k : &tm_v;
+              for (int b = 0; b < C::NBOX; ++b)
+                tma_load_4d(sKV + st * C::TILE_BYTES + b * C::BOX_BYTES, map, bar_kv_full(st), 64 * b, ky,
+                            (int)(kz0 + (int64_t)jt * TC_BN), bh);
+            }
+          }
+        }
+      }
+      // Drain: every load issued must land before the CTA's shared memory goes away.
+      const uint32_t first = use > (uint32_t)C::NSTAGE ? use - C::NSTAGE : 0u;
+      for (uint32_t u = first; u < use; ++u) mbar_wait_drain(bar_kv_full(u % C::NSTAGE), (u / C::NSTAGE) & 1u);
+      mbar_wait_drain(bar_q_full(0), 0);
+      mbar_wait_drain(bar_q_full(1), 0);
+    }
+  } else if (warp == TC_WARP_MMA) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0 && T > 0) {
+      const uint32_t tS[2] = {tmem + C::COL_S0, tmem + C::COL_S1};
+      const uint32_t tO[2] = {tmem + C::COL_O0, tmem + C::COL_O1};
+      auto issue_s = [&](int t, int st) {
+        const uint32_t qa = sQ + t * C::TILE_BYTES;
+        const uint32_t ka = sKV + st * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
+          mma_bf16_ss(tS[t], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), C::IDESC_S,
+                      kk > 0);
+        }
+      };
+      auto issue_pv = [&](int t, int st, bool acc) {
+        const uint32_t va = sKV + st * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < TC_BN / 16; ++kk)
+          mma_bf16_ts(tO[t], tS[t] + kk * 8, sdesc_sw128(va + kk * 2048, C::BOX_BYTES, 1024), C::IDESC_PV,
+                      (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(bar_q_full(0), 0, abort_flag) && mbar_wait(bar_q_full(1), 0, abort_flag);
+      // tile 0: K_0
+      if (ok) ok = mbar_wait(bar_kv_full(0), 0, abort_flag);
+      if (ok) {
+        tc_fence_after_sync();
+        issue_s(0, 0);
+        tc_commit(bar_s_full(0));
+        issue_s(1, 0);
+        tc_commit(bar_s_full(1));
+        tc_commit(bar_kv_empty(0));
+      }
+      for (int n = 1; n < T && ok; ++n) {
+        const uint32_t uv = 2u * (n - 1) + 1u, uk = 2u * n;
+        const int sv = uv % C::NSTAGE, sk = uk % C::NSTAGE;
+        const uint32_t pv = (uv / C::NSTAGE) & 1u, pk = (uk / C::NSTAGE) & 1u;
+        const uint32_t pp = (uint32_t)(n - 1) & 1u;
+        if (!(ok = mbar_wait(bar_kv_full(sv), pv, abort_flag))) break;
+        if (!(ok = mbar_wait(bar_p_full(0), pp, abort_flag))) break;
+        tc_fence_after_sync();
+        issue_pv(0, sv, n - 1 > 0);
+        if (!(ok = mbar_wait(bar_kv_full(sk), pk, abort_flag))) break;
+        tc_fence_after_sync();
+        issue_s(0, sk);
+        tc_commit(bar_s_full(0));
+        if (!(ok = mbar_wait(bar_p_full(1), pp, abort_flag))) break;
+        tc_fence_after_sync();
+        issue_pv(1, sv, n - 1 > 0);
+        tc_commit(bar_kv_empty(sv));
+        issue_s(1, sk);
+        tc_commit(bar_s_full(1));
+        tc_commit(bar_kv_empty(sk));
+      }
+      if (ok) {
+        const uint32_t uv = 2u * (T - 1) + 1u;
+        const int sv = uv % C::NSTAGE;
+        const uint32_t pv = (uv / C::NSTAGE) & 1u, pp = (uint32_t)(T - 1) & 1u;
+        ok = mbar_wait(bar_kv_full(sv), pv, abort_flag) && mbar_wait(bar_p_full(0), pp, abort_flag);
+        if (ok) {
+          tc_fence_after_sync();
+          issue_pv(0, sv, T - 1 > 0);
+          tc_commit(bar_o_done(0));
+          ok = mbar_wait(bar_p_full(1), pp, abort_flag);
+        }
+        if (ok) {
+          tc_fence_after_sync();
+          issue_pv(1, sv, T - 1 > 0);
+          tc_commit(bar_o_done(1));
+          tc_commit(bar_kv_empty(sv));
+        }
+      }
+      // Drain: all MMAs issued by this thread complete before TMEM is released.
+      tc_commit(bar_drain);
+      mbar_wait_drain(bar_drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax warpgroups
+    const int t = warp >> 2;                 // query tile 0 or 1
+    const int row = threadIdx.x & 127;       // row inside the tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + (t == 0 ? C::COL_S0 : C::COL_S1) + lane_off;
+    const uint32_t tO = tmem + (t == 0 ? C::COL_O0 : C::COL_O1) + lane_off;
+    const int64_t li = qb.i0 + (int64_t)t * TC_BM + row;   // local row in the segment
+    const bool row_valid = li < qb.seg.count;
+    const int64_t tq = q_token(pl, qb.seg, li);
+    const int64_t tq_tile_min = q_token(pl, qb.seg, qb.i0 + (int64_t)t * TC_BM);
+    const float sl2 = pl.scale_log2;
+    float m = -INFINITY;   // running max (scaled, log2 units) used for the exponentials
+    float l = 0.f;         // running sum of exp2(s * sl2 - m)
+    int n = 0;
+    bool ok = true;
+    for (int s = 0; s < pl.P && ok; ++s) {
+      int c = qb.p - s;
+      if (c < 0) c += pl.P;
+      for (int sk = 0; sk < nks && ok; ++sk) {
+        const Seg ks = segment_of(pl.layout, pl.P, pl.k_seg_len, c, sk);
+        const int ntiles = (int)((visible_prefix(pl, ks, tq_max) + TC_BN - 1) / TC_BN);
+        const int64_t tks = pl.k_tok_stride * ks.stride;
+        for (int jt = 0; jt < ntiles; ++jt, ++n) {
+          const int64_t j0 = (int64_t)jt * TC_BN;
+          const int vcount = (int)min((int64_t)TC_BN, ks.count - j0);
+          const int64_t tk0 = pl.k_tok0 + pl.k_tok_stride * (ks.row0 + ks.stride * j0);
+          const bool full = vcount == TC_BN && (!pl.causal || tk0 + tks * (TC_BN - 1) <= tq_tile_min);
+          int lim = vcount - 1;  // last visible key of this tile for this row
+          if (pl.causal) {
+            const int64_t jl = tq < tk0 ? -1 : (tq - tk0) / tks;
+            if (jl < lim) lim = (int)jl;
+          }
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(t), (uint32_t)n & 1u, abort_flag))) { ok = false; break; }
+          tc_fence_after_sync();
+          uint32_t sr[TC_BN];
+          RA_TMEM_LD32(tS + 0, (sr + 0));
+          RA_TMEM_LD32(tS + 32, (sr + 32));
+          RA_TMEM_LD32(tS + 64, (sr + 64));
+          RA_TMEM_LD32(tS + 96, (sr + 96));
+          tmem_wait_ld();
+          RA_REG_FENCE32((sr + 0));
+          RA_REG_FENCE32((sr + 32));
+          RA_REG_FENCE32((sr + 64));
+          RA_REG_FENCE32((sr + 96));
+          if (!full) {
+#pragma unroll
+            for (int j = 0; j < TC_BN; ++j) sr[j] = (j <= lim) ? sr[j] : __float_as_uint(-INFINITY);
+          }
+#define SV(j) __uint_as_float(sr[(j)])
+          float mx0 = SV(0), mx1 = SV(1), mx2 = SV(2), mx3 = SV(3);
+#pragma unroll
+          for (int j = 4; j < TC_BN; j += 4) {
+            mx0 = fmaxf(mx0, SV(j));
+            mx1 = fmaxf(mx1, SV(j + 1));
+            mx2 = fmaxf(mx2, SV(j + 2));
+            mx3 = fmaxf(mx3, SV(j + 3));
+          }
+          const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+          // Running max update (conditional rescale, see the file comment).
+          float corr = 1.f;
+          bool rescale = false;
+          if (m == -INFINITY) {
+            m = mx;  // first visible keys of this row: O and l are still 0
+          } else if (mx > m + RESCALE_LOG2) {
+            corr = ex2_approx(m - mx);
+            m = mx;
+            l *= corr;
+            rescale = true;
+          }
+          if (__any_sync(0xffffffffu, rescale) && n > 0) {
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t orr[32];
+              RA_TMEM_LD32(tO + cc * 32, orr);
+              tmem_wait_ld();
+              RA_REG_FENCE32(orr);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * corr);
+              RA_TMEM_ST32(tO + cc * 32, orr);
+            }
+          }
+          const float shift = (m == -INFINITY) ? 0.f : m;
+          float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float p0 = ex2_approx(fmaf(SV(half * 64 + 2 * j), sl2, -shift));
+              const float p1 = ex2_approx(fmaf(SV(half * 64 + 2 * j + 1), sl2, -shift));
+              sum0 += p0;
+              sum1 += p1;
+              pk[j] = pack_bf16x2(p0, p1);
+            }
+            RA_TMEM_ST32(tS + half * 32, pk);
+          }
+#undef SV
+          l += sum0 + sum1;
+          tmem_wait_st();
+          tc_fence_before_sync();
+          mbar_arrive(bar_p_full(t));
+        }
+      }
+    }
+    // ---- epilogue: O = O / l, lse = (m + log2 l) * ln 2
+    if (ok && T > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_o_done(t), 0, abort_flag));
+    if (ok) {
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const int64_t mrow = qb.seg.row0 + qb.seg.stride * li;
+      const int64_t orow = (int64_t)bh * pl.q_rows + mrow;
+      if (T > 0) tc_fence_after_sync();
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t orr[32];
+        if (T > 0) {
+          RA_TMEM_LD32(tO + cc * 32, orr);
+          tmem_wait_ld();
+          RA_REG_FENCE32(orr);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) orr[j] = 0u;
+        }
+        if (row_valid) {
+          if (pl.out_f32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(pl.o) + orow * D + cc * 32);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              dst[j] = make_float4(__uint_as_float(orr[4 * j]) * inv_l, __uint_as_float(orr[4 * j + 1]) * inv_l,
+                                   __uint_as_float(orr[4 * j + 2]) * inv_l, __uint_as_float(orr[4 * j + 3]) * inv_l);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(pl.o) + orow * D + cc * 32);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(orr[8 * j + 0]) * inv_l, __uint_as_float(orr[8 * j + 1]) * inv_l);
+              w.y = pack_bf16x2(__uint_as_float(orr[8 * j + 2]) * inv_l, __uint_as_float(orr[8 * j + 3]) * inv_l);
+              w.z = pack_bf16x2(__uint_as_float(orr[8 * j + 4]) * inv_l, __uint_as_float(orr[8 * j + 5]) * inv_l);
+              w.w = pack_bf16x2(__uint_as_float(orr[8 * j + 6]) * inv_l, __uint_as_float(orr[8 * j + 7]) * inv_l);
+              dst[j] = w;
+            }
+          }
+        }
+      }
+      if (row_valid && pl.lse != nullptr)
+        pl.lse[orow] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+    }
+  }
+
+  // ---- teardown: TMEM is released only after every tcgen05 operation has finished.
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == TC_WARP_MMA) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, TC_TMEM_COLS);
+  }
+}
+
+}  // namespace ra

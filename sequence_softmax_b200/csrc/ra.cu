@@ -1,0 +1,220 @@
+// ra.cu -- libra.so: the C ABI of include/ra.h (argument checks, TMA tensor maps, launch
+// configuration) and the kernels it launches, compiled as one translation unit for sm_100a.
+#include <math.h>
+#include <mutex>
+#include <stdio.h>
+
+#include "common.cuh"
+#include "attn_simt.cuh"
+#include "attn_tc.cuh"
+#include "merge.cuh"
+
+#define RA_ABI_VERSION 1
+
+namespace ra {
+namespace {
+
+// ---- cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda) ----
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 4-D view of a [BH, rows, d] bf16 buffer as (d, S, rows / S, BH): a box of 64 columns x
+// 1 x 128 rows x 1 selects 128 rows spaced S apart (S = P for the striped layout, else 1).
+bool make_tile_map(CUtensorMap* map, const void* base, int BH, int64_t rows, int d, int S) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)S, (cuuint64_t)(rows / S), (cuuint64_t)BH};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)S * d * 2, (cuuint64_t)rows * d * 2};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)TC_BN, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <int D>
+ra_status launch_tc(const Plan& pl, int S, cudaStream_t stream) {
+  using C = TcCfg<D>;
+  CUtensorMap mq, mk, mv;
+  if (!make_tile_map(&mq, pl.q, pl.BH, pl.q_rows, D, S) || !make_tile_map(&mk, pl.k, pl.BH, pl.k_rows, D, S) ||
+      !make_tile_map(&mv, pl.v, pl.BH, pl.k_rows, D, S))
+    return RA_ERR_CUDA;
+  // The dynamic shared-memory opt-in is a per-device function attribute: set it once per device.
+  static bool attr_done[64] = {};
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return RA_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return RA_ERR_UNSUPPORTED;
+    if (!attr_done[dev]) {
+      if (cudaFuncSetAttribute(attn_fwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+          cudaSuccess)
+        return RA_ERR_CUDA;
+      attr_done[dev] = true;
+    }
+  }
+  const int64_t nb = (pl.q_seg_len + 2 * TC_BM - 1) / (2 * TC_BM);
+  const int64_t units = nb * (int64_t)pl.P * num_segments(pl.layout);
+  const int64_t grid = units * pl.BH;
+  if (grid <= 0) return RA_OK;
+  if (grid > 0x7FFFFFFFll) return RA_ERR_UNSUPPORTED;
+  attn_fwd_tc_kernel<D><<<(unsigned)grid, TC_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, pl);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+ra_status launch_attention(const Plan& pl, ra_dtype dt, int S, cudaStream_t stream) {
+  if (dt == RA_BF16) {
+    if (pl.d == 128) return launch_tc<128>(pl, S, stream);
+    if (pl.d == 64) return launch_tc<64>(pl, S, stream);
+    return RA_ERR_UNSUPPORTED;
+  }
+  const int64_t rows_per_pos = pl.q_seg_len * num_segments(pl.layout);
+  const int64_t gx = (rows_per_pos + SIMT_WARPS - 1) / SIMT_WARPS;
+  if (gx <= 0) return RA_OK;
+  if (gx > 0x7FFFFFFFll || pl.P > 65535 || pl.BH > 65535) return RA_ERR_UNSUPPORTED;
+  dim3 grid((unsigned)gx, (unsigned)pl.P, (unsigned)pl.BH);
+  attn_fwd_simt_f32_kernel<<<grid, SIMT_WARPS * 32, 0, stream>>>(pl, rows_per_pos);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+ra_status check_dtype_d(ra_dtype dt, int d) {
+  if (dt != RA_F32 && dt != RA_BF16) return RA_ERR_INVALID_ARG;
+  if (d <= 0) return RA_ERR_INVALID_ARG;
+  if (dt == RA_BF16 && d != 64 && d != 128) return RA_ERR_UNSUPPORTED;
+  if (dt == RA_F32 && d > SIMT_DMAX) return RA_ERR_UNSUPPORTED;
+  return RA_OK;
+}
+
+}  // namespace
+}  // namespace ra
+
+using namespace ra;
+
+extern "C" {
+
+int ra_abi_version(void) { return RA_ABI_VERSION; }
+
+const char* ra_status_string(ra_status s) {
+  switch (s) {
+    case RA_OK: return "RA_OK";
+    case RA_ERR_INVALID_ARG: return "RA_ERR_INVALID_ARG: invalid size, pointer, alignment or enum";
+    case RA_ERR_UNSUPPORTED: return "RA_ERR_UNSUPPORTED: valid but not implemented (dtype / head dim / size)";
+    case RA_ERR_CUDA: return "RA_ERR_CUDA: a CUDA runtime or driver call failed";
+    case RA_ERR_TIMEOUT: return "RA_ERR_TIMEOUT: a bounded wait inside a kernel ran out";
+    case RA_ERR_DEVICE_BOUNDS: return "RA_ERR_DEVICE_BOUNDS: a checked device index was out of range";
+  }
+  return "RA_UNKNOWN_STATUS";
+}
+
+ra_status ra_get_device_error(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return RA_ERR_CUDA;
+  unsigned word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return RA_ERR_CUDA;
+  if (word != 0) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return RA_ERR_CUDA;
+  }
+  if (word & DEVERR_TIMEOUT) return RA_ERR_TIMEOUT;
+  if (word & DEVERR_BOUNDS) return RA_ERR_DEVICE_BOUNDS;
+  return RA_OK;
+}
+
+ra_status ra_partial(const void* q, const void* k, const void* v, ra_dtype dt, int B, int H, int64_t Lq,
+                     int64_t Lk, int d, float scale, int causal, int64_t q_tok0, int64_t q_tok_stride,
+                     int64_t k_tok0, int64_t k_tok_stride, float* o_partial, float* lse, cudaStream_t stream) {
+  if (B < 0 || H < 0 || Lq < 0 || Lk < 0) return RA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return RA_ERR_INVALID_ARG;
+  if (q_tok_stride < 1 || k_tok_stride < 1) return RA_ERR_INVALID_ARG;
+  ra_status st = check_dtype_d(dt, d);
+  if (st != RA_OK) return st;
+  if ((int64_t)B * H > 0x7FFFFFFF) return RA_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || Lq == 0) return RA_OK;
+  if (!q || !o_partial || !lse || !aligned16(q) || !aligned16(o_partial) || !aligned16(lse)) return RA_ERR_INVALID_ARG;
+  if (Lk == 0) {
+    const int64_t rows = (int64_t)B * H * Lq;
+    fill_empty_kernel<<<592, 256, 0, stream>>>(o_partial, lse, rows, d);
+    return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+  }
+  if (!k || !v || !aligned16(k) || !aligned16(v)) return RA_ERR_INVALID_ARG;
+  Plan pl{};
+  pl.q = q; pl.k = k; pl.v = v; pl.o = o_partial; pl.lse = lse;
+  pl.BH = B * H; pl.d = d; pl.P = 1; pl.layout = RA_LAYOUT_CONTIGUOUS; pl.causal = causal; pl.out_f32 = 1;
+  pl.q_rows = Lq; pl.k_rows = Lk; pl.q_seg_len = Lq; pl.k_seg_len = Lk;
+  pl.q_tok0 = q_tok0; pl.q_tok_stride = q_tok_stride; pl.k_tok0 = k_tok0; pl.k_tok_stride = k_tok_stride;
+  pl.scale = scale;
+  pl.scale_log2 = scale * 1.4426950408889634f;
+  return launch_attention(pl, dt, 1, stream);
+}
+
+ra_status ra_merge(const float* o_parts, const float* lse_parts, int n, int64_t rows, int d, void* o_out,
+                   ra_dtype out_dt, float* lse_out, cudaStream_t stream) {
+  if (n < 1 || rows < 0 || d < 1 || (d & 3) != 0) return RA_ERR_INVALID_ARG;
+  if (out_dt != RA_F32 && out_dt != RA_BF16) return RA_ERR_INVALID_ARG;
+  if (n > MERGE_MAX_PARTS) return RA_ERR_UNSUPPORTED;
+  if (rows == 0) return RA_OK;
+  if (!o_parts || !lse_parts || !o_out || !aligned16(o_parts) || !aligned16(o_out)) return RA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(lse_parts) & 3u) || (lse_out && (reinterpret_cast<uintptr_t>(lse_out) & 3u)))
+    return RA_ERR_INVALID_ARG;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t warps_needed = (rows + 1) / 2;
+  int64_t blocks = (warps_needed * 32 + MERGE_THREADS - 1) / MERGE_THREADS;
+  const int64_t cap = (int64_t)sms * 8;  // 8 resident blocks of 256 threads per SM
+  if (blocks > cap) blocks = cap;
+  if (out_dt == RA_BF16)
+    merge_kernel<true><<<(unsigned)blocks, MERGE_THREADS, 0, stream>>>(o_parts, lse_parts, n, rows, d, o_out, lse_out);
+  else
+    merge_kernel<false><<<(unsigned)blocks, MERGE_THREADS, 0, stream>>>(o_parts, lse_parts, n, rows, d, o_out, lse_out);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+ra_status ra_ring_forward(const void* q, const void* k, const void* v, ra_dtype dt, int B, int H, int64_t N, int d,
+                          float scale, int n_chunks, int causal, ra_layout layout, void* o, float* lse,
+                          cudaStream_t stream) {
+  if (B < 0 || H < 0 || N < 0 || n_chunks < 1) return RA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return RA_ERR_INVALID_ARG;
+  if (layout != RA_LAYOUT_CONTIGUOUS && layout != RA_LAYOUT_STRIPED && layout != RA_LAYOUT_ZIGZAG)
+    return RA_ERR_INVALID_ARG;
+  const int64_t parts = layout == RA_LAYOUT_ZIGZAG ? 2 * (int64_t)n_chunks : n_chunks;
+  if (N % parts != 0) return RA_ERR_INVALID_ARG;
+  ra_status st = check_dtype_d(dt, d);
+  if (st != RA_OK) return st;
+  if ((int64_t)B * H > 0x7FFFFFFF) return RA_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || N == 0) return RA_OK;
+  if (!q || !k || !v || !o || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return RA_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return RA_ERR_INVALID_ARG;
+  Plan pl{};
+  pl.q = q; pl.k = k; pl.v = v; pl.o = o; pl.lse = lse;
+  pl.BH = B * H; pl.d = d; pl.P = n_chunks; pl.layout = layout; pl.causal = causal; pl.out_f32 = (dt == RA_F32);
+  pl.q_rows = N; pl.k_rows = N;
+  pl.q_seg_len = pl.k_seg_len = N / parts;
+  pl.q_tok0 = 0; pl.q_tok_stride = 1; pl.k_tok0 = 0; pl.k_tok_stride = 1;
+  pl.scale = scale;
+  pl.scale_log2 = scale * 1.4426950408889634f;
+  const int S = layout == RA_LAYOUT_STRIPED ? n_chunks : 1;
+  return launch_attention(pl, dt, S, stream);
+}
+
+}  // extern "C"

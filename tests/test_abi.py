@@ -1,0 +1,136 @@
+"""The C-ABI library on a host without a GPU: it builds, loads, exports every symbol that
+include/ra.h declares, and rejects invalid arguments with status codes before touching
+the device (no compute call is made here)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from sequence_softmax_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ra.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ra_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for name in ("ra_partial", "ra_merge", "ra_ring_forward", "ra_status_string", "ra_get_device_error"):
+        assert name in syms
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert set(declared_symbols()) == set(binding.SIGNATURES)
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.ra_abi_version() == 1
+    for code in range(6):
+        s = binding.status_string(code)
+        assert s.startswith("RA_")
+    assert binding.status_string(99) == "RA_UNKNOWN_STATUS"
+
+
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every call below fails validation first
+
+
+def _ring(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, dt=1, B=1, H=1, N=256, d=128, scale=0.1, n_chunks=2, causal=1,
+             layout=0, o=FAKE, lse=None, stream=None)
+    a.update(kw)
+    return lib.ra_ring_forward(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_chunks=0), binding.RA_ERR_INVALID_ARG),
+    (dict(N=250, n_chunks=4), binding.RA_ERR_INVALID_ARG),            # N % P != 0
+    (dict(N=256, n_chunks=3, layout=2), binding.RA_ERR_INVALID_ARG),  # zig-zag needs N % 2P == 0
+    (dict(layout=7), binding.RA_ERR_INVALID_ARG),
+    (dict(scale=0.0), binding.RA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), binding.RA_ERR_INVALID_ARG),
+    (dict(causal=2), binding.RA_ERR_INVALID_ARG),
+    (dict(dt=5), binding.RA_ERR_INVALID_ARG),
+    (dict(d=96), binding.RA_ERR_UNSUPPORTED),                         # bf16 needs d in {64, 128}
+    (dict(dt=0, d=160), binding.RA_ERR_UNSUPPORTED),                  # fp32 needs d <= 128
+    (dict(B=-1), binding.RA_ERR_INVALID_ARG),
+    (dict(q=ctypes.c_void_p(0x10008)), binding.RA_ERR_INVALID_ARG),  # 8-byte aligned only
+    (dict(o=None), binding.RA_ERR_INVALID_ARG),
+])
+def test_ring_forward_rejects(lib, kw, code):
+    assert _ring(lib, **kw) == code
+
+
+def test_ring_forward_empty_is_noop(lib):
+    assert _ring(lib, N=0) == binding.RA_OK
+    assert _ring(lib, B=0) == binding.RA_OK
+    assert _ring(lib, H=0) == binding.RA_OK
+
+
+def _partial(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, dt=1, B=1, H=1, Lq=128, Lk=128, d=64, scale=0.1, causal=0,
+             q_tok0=0, q_ts=1, k_tok0=0, k_ts=1, o=FAKE, lse=FAKE, stream=None)
+    a.update(kw)
+    return lib.ra_partial(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Lq=-1), binding.RA_ERR_INVALID_ARG),
+    (dict(q_ts=0), binding.RA_ERR_INVALID_ARG),
+    (dict(k_ts=-2), binding.RA_ERR_INVALID_ARG),
+    (dict(d=32), binding.RA_ERR_UNSUPPORTED),
+    (dict(lse=None), binding.RA_ERR_INVALID_ARG),
+    (dict(scale=-1.0), binding.RA_ERR_INVALID_ARG),
+])
+def test_partial_rejects(lib, kw, code):
+    assert _partial(lib, **kw) == code
+
+
+def test_partial_empty_is_noop(lib):
+    assert _partial(lib, Lq=0) == binding.RA_OK
+
+
+def _merge(lib, **kw):
+    a = dict(o=FAKE, lse=FAKE, n=2, rows=16, d=128, out=FAKE, out_dt=1, lse_out=None, stream=None)
+    a.update(kw)
+    return lib.ra_merge(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n=0), binding.RA_ERR_INVALID_ARG),
+    (dict(d=6), binding.RA_ERR_INVALID_ARG),       # d % 4 != 0
+    (dict(out_dt=3), binding.RA_ERR_INVALID_ARG),
+    (dict(n=65), binding.RA_ERR_UNSUPPORTED),
+    (dict(rows=-1), binding.RA_ERR_INVALID_ARG),
+    (dict(out=None), binding.RA_ERR_INVALID_ARG),
+])
+def test_merge_rejects(lib, kw, code):
+    assert _merge(lib, **kw) == code
+
+
+def test_merge_empty_is_noop(lib):
+    assert _merge(lib, rows=0) == binding.RA_OK
+
+
+def test_product_path_does_not_reach_the_oracle():
+    """The CUDA path's sources never import or link the CPU oracle."""
+    pkg = os.path.join(ROOT, "sequence_softmax_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f

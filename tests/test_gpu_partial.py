@@ -1,0 +1,65 @@
+"""ra_partial on the GPU against the oracle's partial state (fp64), through the C-ABI."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sequence_softmax_b200 import binding
+from sequence_softmax_b200.inputs import make_qkv
+
+from .parity import compare, to_np
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    # dtype, B, H, Lq, Lk, d, causal, q_tok0, q_ts, k_tok0, k_ts
+    ("f32", 1, 2, 64, 96, 16, False, 0, 1, 0, 1),
+    ("f32", 2, 1, 70, 45, 128, True, 100, 1, 60, 1),      # ragged, partly visible
+    ("f32", 1, 1, 40, 40, 33, True, 3, 4, 1, 4),          # striped positions
+    ("bf16", 1, 2, 256, 256, 128, False, 0, 1, 0, 1),
+    ("bf16", 2, 2, 384, 640, 64, False, 0, 1, 0, 1),
+    ("bf16", 1, 3, 300, 333, 128, False, 0, 1, 0, 1),     # ragged tails on both sides
+    ("bf16", 1, 2, 512, 512, 128, True, 512, 1, 0, 1),    # chunk wholly in the past: full
+    ("bf16", 1, 2, 512, 512, 128, True, 0, 1, 0, 1),      # diagonal chunk
+    ("bf16", 1, 2, 512, 512, 64, True, 0, 1, 256, 1),     # keys partly in the future, empty rows
+    ("bf16", 1, 1, 256, 256, 128, True, 0, 1, 4096, 1),   # keys wholly in the future: all empty
+    ("bf16", 1, 2, 256, 384, 128, True, 5, 16, 2, 16),    # striped query / key positions
+    ("bf16", 1, 1, 1, 1, 128, False, 0, 1, 0, 1),         # one row, one key
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "-".join(map(str, c)))
+def test_partial_matches_oracle(cuda, case):
+    kind, B, H, Lq, Lk, d, causal, qt0, qts, kt0, kts = case
+    dtype = torch.float32 if kind == "f32" else torch.bfloat16
+    q, _, _ = make_qkv(B, H, Lq, d, dtype, seed=Lq + Lk, device="cuda")
+    _, k, v = make_qkv(B, H, Lk, d, dtype, seed=Lq * Lk + 1, device="cuda")
+    o, lse = binding.partial(q, k, v, causal=causal, q_tok0=qt0, q_tok_stride=qts, k_tok0=kt0, k_tok_stride=kts)
+    assert binding.get_device_error() == binding.RA_OK
+    o_ref, lse_ref = oracle.partial(to_np(q), to_np(k), to_np(v), d ** -0.5, causal, qt0, qts, kt0, kts)
+    compare(to_np(o), to_np(lse), o_ref, lse_ref, kind, str(case))
+
+
+def test_partial_empty_keys(cuda):
+    q, _, _ = make_qkv(1, 2, 100, 128, torch.bfloat16, seed=1, device="cuda")
+    k = torch.empty(1, 2, 0, 128, device="cuda", dtype=torch.bfloat16)
+    o, lse = binding.partial(q, k, k.clone())
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_partials_merge_to_full_attention(cuda):
+    """The ring's arithmetic in pieces: partial states of 4 KV chunks merged on the GPU equal
+    full causal attention from the oracle."""
+    B, H, N, d, P = 1, 2, 1024, 128, 4
+    q, k, v = make_qkv(B, H, N, d, torch.bfloat16, seed=11, device="cuda")
+    c = N // P
+    parts_o, parts_l = [], []
+    for p in range(P):
+        o_p, l_p = binding.partial(q, k[:, :, p * c:(p + 1) * c].contiguous(), v[:, :, p * c:(p + 1) * c].contiguous(),
+                                   causal=True, q_tok0=0, q_tok_stride=1, k_tok0=p * c, k_tok_stride=1)
+        parts_o.append(o_p)
+        parts_l.append(l_p)
+    out, L = binding.merge(torch.stack(parts_o), torch.stack(parts_l), out_dtype=torch.bfloat16)
+    o_ref, l_ref = oracle.attention(to_np(q), to_np(k), to_np(v), d ** -0.5, True)
+    compare(to_np(out), to_np(L), o_ref, l_ref, "bf16", "partials+merge")
