@@ -71,7 +71,11 @@ merge_kernel(const float* __restrict__ o_parts, const float* __restrict__ lse_pa
       w[q][1] = e1 * inv;
       L[q] = tot > 0.f ? sh + logf(tot) : -INFINITY;
     }
-    for (int c = lane; c < d4; c += 32) {
+    // Uniform trip count so that every lane takes part in the weight shuffles.
+    for (int c0 = 0; c0 < d4; c0 += 32) {
+      const int c = c0 + lane;
+      const bool act = c < d4;
+      const int cc = act ? c : 0;  // inactive lanes read a valid address and store nothing
       float4 acc[2];
       acc[0] = make_float4(0.f, 0.f, 0.f, 0.f);
       acc[1] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -79,12 +83,12 @@ merge_kernel(const float* __restrict__ o_parts, const float* __restrict__ lse_pa
       for (; i + 2 <= n; i += 2) {
         const float wa0 = weight_of(w[0], i), wb0 = weight_of(w[0], i + 1);
         const float wa1 = weight_of(w[1], i), wb1 = weight_of(w[1], i + 1);
-        const float4 a0 = __ldcs(op4 + i * part_stride4 + r0 * d4 + c);
-        const float4 b0 = __ldcs(op4 + (i + 1) * part_stride4 + r0 * d4 + c);
+        const float4 a0 = __ldcs(op4 + i * part_stride4 + r0 * d4 + cc);
+        const float4 b0 = __ldcs(op4 + (i + 1) * part_stride4 + r0 * d4 + cc);
         float4 a1 = make_float4(0.f, 0.f, 0.f, 0.f), b1 = a1;
         if (nr == 2) {
-          a1 = __ldcs(op4 + i * part_stride4 + (r0 + 1) * d4 + c);
-          b1 = __ldcs(op4 + (i + 1) * part_stride4 + (r0 + 1) * d4 + c);
+          a1 = __ldcs(op4 + i * part_stride4 + (r0 + 1) * d4 + cc);
+          b1 = __ldcs(op4 + (i + 1) * part_stride4 + (r0 + 1) * d4 + cc);
         }
         acc[0].x = fmaf(wa0, a0.x, fmaf(wb0, b0.x, acc[0].x));
         acc[0].y = fmaf(wa0, a0.y, fmaf(wb0, b0.y, acc[0].y));
@@ -97,9 +101,9 @@ merge_kernel(const float* __restrict__ o_parts, const float* __restrict__ lse_pa
       }
       for (; i < n; ++i) {
         const float wa0 = weight_of(w[0], i), wa1 = weight_of(w[1], i);
-        const float4 a0 = __ldcs(op4 + i * part_stride4 + r0 * d4 + c);
+        const float4 a0 = __ldcs(op4 + i * part_stride4 + r0 * d4 + cc);
         float4 a1 = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (nr == 2) a1 = __ldcs(op4 + i * part_stride4 + (r0 + 1) * d4 + c);
+        if (nr == 2) a1 = __ldcs(op4 + i * part_stride4 + (r0 + 1) * d4 + cc);
         acc[0].x = fmaf(wa0, a0.x, acc[0].x);
         acc[0].y = fmaf(wa0, a0.y, acc[0].y);
         acc[0].z = fmaf(wa0, a0.z, acc[0].z);
@@ -109,8 +113,10 @@ merge_kernel(const float* __restrict__ o_parts, const float* __restrict__ lse_pa
         acc[1].z = fmaf(wa1, a1.z, acc[1].z);
         acc[1].w = fmaf(wa1, a1.w, acc[1].w);
       }
-      merge_store4<OUT_BF16>(o_out, r0 * d4 + c, acc[0].x, acc[0].y, acc[0].z, acc[0].w);
-      if (nr == 2) merge_store4<OUT_BF16>(o_out, (r0 + 1) * d4 + c, acc[1].x, acc[1].y, acc[1].z, acc[1].w);
+      if (act) {
+        merge_store4<OUT_BF16>(o_out, r0 * d4 + c, acc[0].x, acc[0].y, acc[0].z, acc[0].w);
+        if (nr == 2) merge_store4<OUT_BF16>(o_out, (r0 + 1) * d4 + c, acc[1].x, acc[1].y, acc[1].z, acc[1].w);
+      }
     }
     if (lse_out != nullptr && lane == 0) {
       lse_out[r0] = L[0];
