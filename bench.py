@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-merge", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--merge-rows", type=int, default=8 * (1 << 20),
+                    help="rows of the merge workload (smaller values for profiler captures)")
     return ap.parse_args()
 
 
@@ -321,7 +323,7 @@ def main():
 
 def bench_merge(binding, torch, dev, pk, a):
     """ra_merge on 2 fp32 partial states shaped like the 1M-token workload -> bf16 O + fp32 lse."""
-    n, rows, d = 2, 8 * (1 << 20), 128
+    n, rows, d = 2, a.merge_rows, 128
     g = torch.Generator(device=dev).manual_seed(99)
     o_parts = torch.randn(n, rows, d, device=dev, generator=g)
     lse_parts = torch.randn(n, rows, device=dev, generator=g) + 10.0
@@ -340,7 +342,7 @@ def bench_merge(binding, torch, dev, pk, a):
     ms = s.elapsed_time(e) / iters
     nbytes = n * rows * (4 * d + 4) + rows * (2 * d + 4)
     gbs = nbytes / (ms / 1e3) / 1e9
-    traffic = stored_traffic("merge", "merge-n2-rows8M-d128", rows)
+    traffic = stored_traffic("merge", f"merge-n2-rows{rows}-d128", rows)
     return {"value": gbs, "unit": "GB/s", "ms": ms, "bytes": nbytes, "launches": iters,
             "workload": f"n={n} fp32 partials, rows={rows}, d={d} -> bf16 O + fp32 lse",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",

@@ -7,7 +7,7 @@
 // [CARD] online softmax). Causal tiles wholly in the future are never visited; tiles that
 // straddle the diagonal are masked elementwise ([BLOG] ring_attention_causal_step).
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads, 3 warpgroups; setmaxnreg moves registers to the softmax):
 //   warps 0-3  softmax for query tile 0 (thread i owns row i = TMEM lane i)
 //   warps 4-7  softmax for query tile 1
 //   warp  8    TMA producer: Q tiles once, then K/V tiles into an NSTAGE ring of shared
@@ -15,6 +15,7 @@
 //              chunk's transfer with the current chunk's compute)
 //   warp  9    MMA issuer (one thread): S_t = Q_t K^T (both operands from 128B-swizzled
 //              shared memory) and O_t += P_t V (P from tensor memory, V from shared memory)
+//   warps 10-11 idle
 //
 // Tensor memory (512 columns x 128 lanes of fp32): S_0 | S_1 | O_0 | O_1. P_t (bf16 pairs)
 // overwrites the first 64 columns of S_t. The MMA warp issues, per KV tile n,
@@ -36,7 +37,9 @@ namespace ra {
 
 constexpr int TC_BM = 128;          // query rows per tile
 constexpr int TC_BN = 128;          // keys per KV tile
-constexpr int TC_THREADS = 320;
+constexpr int TC_THREADS = 384;     // 3 warpgroups
+constexpr int TC_REGS_SOFTMAX = 216;  // per thread, after setmaxnreg (launch: 168)
+constexpr int TC_REGS_OTHER = 72;     // 2 x 216 + 72 = 504 = 168 * 384 / 128
 constexpr int TC_WARP_PRODUCER = 8;
 constexpr int TC_WARP_MMA = 9;
 constexpr int TC_TMEM_COLS = 512;
@@ -91,6 +94,76 @@ __device__ __forceinline__ QBlock decode_unit(const Plan& pl, int unit) {
 
 __device__ __forceinline__ int64_t q_token(const Plan& pl, const Seg& s, int64_t i) {
   return pl.q_tok0 + pl.q_tok_stride * (s.row0 + s.stride * i);
+}
+
+// exp2 on the FMA pipe for a share of the scores, so that the MUFU (16 results per SM
+// per clock) and the FMA pipes share the softmax's exponentials. Cody-Waite reduction
+// 2^x = 2^round(x) * 2^f, f in [-1/2, 1/2], with the degree-3 minimax polynomial printed by
+// csrc/exp2_poly.py (Remez exchange; max relative error 7.5e-5, far below bf16's 2^-9).
+// round(x) comes from adding and subtracting 1.5 * 2^23; 2^n is added into the exponent
+// field. x is clamped to >= -126 so that the exponent never wraps; 2^-126 is below any
+// visible contribution (the row max contributes >= 1).
+constexpr float EXP2_C0 = 9.999280735e-01f, EXP2_C1 = 6.932609855e-01f, EXP2_C2 = 2.426111222e-01f,
+                EXP2_C3 = 5.517166906e-02f;
+constexpr float ROUND_MAGIC = 12582912.0f;  // 1.5 * 2^23
+// Pairs of scores per group of 8 pairs that take the FMA-pipe exp2 (the rest use MUFU).
+#ifndef RA_EMU_PAIRS_OF_8
+#define RA_EMU_PAIRS_OF_8 0
+#endif
+
+__device__ __forceinline__ void exp2_poly_pair(uint64_t x2, float& p0, float& p1) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  x2 = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t2 = f2_add(x2, f2_pack(ROUND_MAGIC, ROUND_MAGIC));
+  const uint64_t n2 = f2_add(t2, f2_pack(-ROUND_MAGIC, -ROUND_MAGIC));
+  const uint64_t f2 = f2_fma(n2, f2_pack(-1.f, -1.f), x2);
+  uint64_t q2 = f2_fma(f2_pack(EXP2_C3, EXP2_C3), f2, f2_pack(EXP2_C2, EXP2_C2));
+  q2 = f2_fma(q2, f2, f2_pack(EXP2_C1, EXP2_C1));
+  q2 = f2_fma(q2, f2, f2_pack(EXP2_C0, EXP2_C0));
+  float q0, q1, t0, t1;
+  f2_unpack(q2, q0, q1);
+  f2_unpack(t2, t0, t1);
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
+// P = exp2(s * sl2 - shift) for one row of 128 scores: writes P as bf16 pairs into TMEM
+// columns [0, 64) at tS and returns the row sums of the even and odd columns. With EMU,
+// RA_EMU_PAIRS_OF_8 pairs in eight go through exp2_poly_pair (only on tiles without
+// masked scores).
+template <bool EMU>
+__device__ __forceinline__ void exp_tile(const uint32_t (&sr)[TC_BN], float sl2, float shift, uint32_t tS,
+                                         float& sum0, float& sum1) {
+  const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-shift, -shift);
+  uint64_t sum2a = f2_pack(0.f, 0.f), sum2b = sum2a;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[half * 64 + 2 * j]),
+                                         __uint_as_float(sr[half * 64 + 2 * j + 1])), sl2x2, negm2);
+      float p0, p1;
+      if (EMU && (j & 7) >= 8 - RA_EMU_PAIRS_OF_8) {
+        exp2_poly_pair(x2, p0, p1);
+      } else {
+        float x0, x1;
+        f2_unpack(x2, x0, x1);
+        p0 = ex2_approx(x0);
+        p1 = ex2_approx(x1);
+      }
+      if (j & 1) sum2b = f2_add(sum2b, f2_pack(p0, p1));
+      else sum2a = f2_add(sum2a, f2_pack(p0, p1));
+      pk[j] = pack_bf16x2(p0, p1);
+    }
+    RA_TMEM_ST32(tS + half * 32, pk);
+  }
+  float sa0, sa1, sb0, sb1;
+  f2_unpack(sum2a, sa0, sa1);
+  f2_unpack(sum2b, sb0, sb1);
+  sum0 = sa0 + sb0;
+  sum1 = sa1 + sb1;
 }
 
 template <int D>
@@ -164,6 +237,10 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
   }
 
+  if (warp >= 8) {
+    // Warpgroup 2 (TMA producer, MMA issuer, two idle warps) gives registers to the softmax.
+    regs_decrease<TC_REGS_OTHER>();
+  }
   if (warp == TC_WARP_PRODUCER) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -207,7 +284,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
   } else if (warp == TC_WARP_MMA) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0 && T > 0) {
+    // The whole warp runs the loop (converged) and one elected lane issues: tcgen05.mma
+    // issued from a converged warp streams much faster than from a lone diverged thread.
+    if (T > 0) {
       const uint32_t tS[2] = {tmem + C::COL_S0, tmem + C::COL_S1};
       const uint32_t tO[2] = {tmem + C::COL_O0, tmem + C::COL_O1};
       auto issue_s = [&](int t, int st) {
@@ -227,62 +306,85 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           mma_bf16_ts(tO[t], tS[t] + kk * 8, sdesc_sw128(va + kk * 2048, C::BOX_BYTES, 1024), C::IDESC_PV,
                       (acc || kk > 0) ? 1u : 0u);
       };
-      bool ok = mbar_wait(bar_q_full(0), 0, abort_flag) && mbar_wait(bar_q_full(1), 0, abort_flag);
+      auto wait_all = [&](uint32_t bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+      };
+      bool ok = wait_all(bar_q_full(0), 0) && wait_all(bar_q_full(1), 0);
       // tile 0: K_0
-      if (ok) ok = mbar_wait(bar_kv_full(0), 0, abort_flag);
+      if (ok) ok = wait_all(bar_kv_full(0), 0);
       if (ok) {
         tc_fence_after_sync();
-        issue_s(0, 0);
-        tc_commit(bar_s_full(0));
-        issue_s(1, 0);
-        tc_commit(bar_s_full(1));
-        tc_commit(bar_kv_empty(0));
+        if (elect_one()) {
+          issue_s(0, 0);
+          tc_commit(bar_s_full(0));
+          issue_s(1, 0);
+          tc_commit(bar_s_full(1));
+          tc_commit(bar_kv_empty(0));
+        }
+        __syncwarp();
       }
       for (int n = 1; n < T && ok; ++n) {
         const uint32_t uv = 2u * (n - 1) + 1u, uk = 2u * n;
         const int sv = uv % C::NSTAGE, sk = uk % C::NSTAGE;
         const uint32_t pv = (uv / C::NSTAGE) & 1u, pk = (uk / C::NSTAGE) & 1u;
         const uint32_t pp = (uint32_t)(n - 1) & 1u;
-        if (!(ok = mbar_wait(bar_kv_full(sv), pv, abort_flag))) break;
-        if (!(ok = mbar_wait(bar_p_full(0), pp, abort_flag))) break;
+        if (!(ok = wait_all(bar_kv_full(sv), pv))) break;
+        if (!(ok = wait_all(bar_p_full(0), pp))) break;
         tc_fence_after_sync();
-        issue_pv(0, sv, n - 1 > 0);
-        if (!(ok = mbar_wait(bar_kv_full(sk), pk, abort_flag))) break;
+        if (elect_one()) issue_pv(0, sv, n - 1 > 0);
+        __syncwarp();
+        if (!(ok = wait_all(bar_kv_full(sk), pk))) break;
         tc_fence_after_sync();
-        issue_s(0, sk);
-        tc_commit(bar_s_full(0));
-        if (!(ok = mbar_wait(bar_p_full(1), pp, abort_flag))) break;
+        if (elect_one()) {
+          issue_s(0, sk);
+          tc_commit(bar_s_full(0));
+        }
+        __syncwarp();
+        if (!(ok = wait_all(bar_p_full(1), pp))) break;
         tc_fence_after_sync();
-        issue_pv(1, sv, n - 1 > 0);
-        tc_commit(bar_kv_empty(sv));
-        issue_s(1, sk);
-        tc_commit(bar_s_full(1));
-        tc_commit(bar_kv_empty(sk));
+        if (elect_one()) {
+          issue_pv(1, sv, n - 1 > 0);
+          tc_commit(bar_kv_empty(sv));
+          issue_s(1, sk);
+          tc_commit(bar_s_full(1));
+          tc_commit(bar_kv_empty(sk));
+        }
+        __syncwarp();
       }
       if (ok) {
         const uint32_t uv = 2u * (T - 1) + 1u;
         const int sv = uv % C::NSTAGE;
         const uint32_t pv = (uv / C::NSTAGE) & 1u, pp = (uint32_t)(T - 1) & 1u;
-        ok = mbar_wait(bar_kv_full(sv), pv, abort_flag) && mbar_wait(bar_p_full(0), pp, abort_flag);
+        ok = wait_all(bar_kv_full(sv), pv) && wait_all(bar_p_full(0), pp);
         if (ok) {
           tc_fence_after_sync();
-          issue_pv(0, sv, T - 1 > 0);
-          tc_commit(bar_o_done(0));
-          ok = mbar_wait(bar_p_full(1), pp, abort_flag);
+          if (elect_one()) {
+            issue_pv(0, sv, T - 1 > 0);
+            tc_commit(bar_o_done(0));
+          }
+          __syncwarp();
+          ok = wait_all(bar_p_full(1), pp);
         }
         if (ok) {
           tc_fence_after_sync();
-          issue_pv(1, sv, T - 1 > 0);
-          tc_commit(bar_o_done(1));
-          tc_commit(bar_kv_empty(sv));
+          if (elect_one()) {
+            issue_pv(1, sv, T - 1 > 0);
+            tc_commit(bar_o_done(1));
+            tc_commit(bar_kv_empty(sv));
+          }
+          __syncwarp();
         }
       }
-      // Drain: all MMAs issued by this thread complete before TMEM is released.
-      tc_commit(bar_drain);
-      mbar_wait_drain(bar_drain, 0);
+      // Drain: all MMAs issued by the elected lane complete before TMEM is released.
+      if (elect_one()) {
+        tc_commit(bar_drain);
+        mbar_wait_drain(bar_drain, 0);
+      }
+      __syncwarp();
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------------ softmax warpgroups
+    regs_increase<TC_REGS_SOFTMAX>();
     const int t = warp >> 2;                 // query tile 0 or 1
     const int row = threadIdx.x & 127;       // row inside the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -331,14 +433,17 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             for (int j = 0; j < TC_BN; ++j) sr[j] = (j <= lim) ? sr[j] : __float_as_uint(-INFINITY);
           }
 #define SV(j) __uint_as_float(sr[(j)])
-          float mx0 = SV(0), mx1 = SV(1), mx2 = SV(2), mx3 = SV(3);
+          float mx0 = fmax3(SV(0), SV(1), SV(2)), mx1 = fmax3(SV(3), SV(4), SV(5));
+          float mx2 = fmax3(SV(6), SV(7), SV(8)), mx3 = fmax3(SV(9), SV(10), SV(11));
 #pragma unroll
-          for (int j = 4; j < TC_BN; j += 4) {
-            mx0 = fmaxf(mx0, SV(j));
-            mx1 = fmaxf(mx1, SV(j + 1));
-            mx2 = fmaxf(mx2, SV(j + 2));
-            mx3 = fmaxf(mx3, SV(j + 3));
+          for (int j = 12; j < TC_BN - 8; j += 8) {
+            mx0 = fmax3(mx0, SV(j), SV(j + 1));
+            mx1 = fmax3(mx1, SV(j + 2), SV(j + 3));
+            mx2 = fmax3(mx2, SV(j + 4), SV(j + 5));
+            mx3 = fmax3(mx3, SV(j + 6), SV(j + 7));
           }
+          mx0 = fmax3(mx0, SV(TC_BN - 4), SV(TC_BN - 3));
+          mx1 = fmax3(mx1, SV(TC_BN - 2), SV(TC_BN - 1));
           const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
           // Running max update (conditional rescale, see the file comment).
           float corr = 1.f;
@@ -364,20 +469,11 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
           }
           const float shift = (m == -INFINITY) ? 0.f : m;
-          float sum0 = 0.f, sum1 = 0.f;
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t pk[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float p0 = ex2_approx(fmaf(SV(half * 64 + 2 * j), sl2, -shift));
-              const float p1 = ex2_approx(fmaf(SV(half * 64 + 2 * j + 1), sl2, -shift));
-              sum0 += p0;
-              sum1 += p1;
-              pk[j] = pack_bf16x2(p0, p1);
-            }
-            RA_TMEM_ST32(tS + half * 32, pk);
-          }
+          float sum0, sum1;
+          if (full)
+            exp_tile<true>(sr, sl2, shift, tS, sum0, sum1);
+          else
+            exp_tile<false>(sr, sl2, shift, tS, sum0, sum1);
 #undef SV
           l += sum0 + sum1;
           tmem_wait_st();
