@@ -33,8 +33,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "ring-attn fwd TFLOP/s (bf16, 1 B200), % of tensor peak; merge HBM GB/s"
 PROFILE_JSON = os.path.join(ROOT, "profiles", "counters.json")
-KERNEL_SOURCES = ["sequence_softmax_b200/csrc/attn_tc.cuh", "sequence_softmax_b200/csrc/common.cuh",
-                  "sequence_softmax_b200/csrc/merge.cuh"]
+KERNEL_SOURCES = {
+    "attn_fwd_tc": ["sequence_softmax_b200/csrc/attn_tc.cuh", "sequence_softmax_b200/csrc/common.cuh"],
+    "merge": ["sequence_softmax_b200/csrc/merge.cuh", "sequence_softmax_b200/csrc/common.cuh"],
+}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "source": "fallback"}
 
@@ -65,9 +67,10 @@ def peaks():
     return dict(FALLBACK_PEAKS)
 
 
-def kernel_src_sha() -> str:
+def kernel_src_sha(kernel: str) -> str:
+    """Hash of the sources a kernel is built from (stored next to its ncu counters)."""
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -80,7 +83,7 @@ def stored_traffic(kernel: str, workload: str, units: float):
     with open(PROFILE_JSON) as f:
         prof = json.load(f)
     e = prof.get(kernel)
-    if not e or e.get("kernel_src_sha") != kernel_src_sha():
+    if not e or e.get("kernel_src_sha") != kernel_src_sha(kernel):
         return None
     # traffic per unit processed in the captured case, scaled to this launch's units
     return e["dram_bytes"] / e["units"] * units if e.get("workload") != workload else e["dram_bytes"]
@@ -212,6 +215,17 @@ def run_reference(a, w):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The slowest rank's time: every rank contributes its own CUDA-event time."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def workload_config(w):
     return {"workload": w.name, "batch": w.B, "heads": w.H, "seq_len": w.N, "head_dim": w.d,
             "causal": w.causal, "layout": w.layout, "n_chunks": w.n_chunks, "emit_lse": w.emit_lse,
@@ -273,11 +287,7 @@ def main():
             step()
         end.record(stream)
         barrier()
-    ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end), world, dev)
     if binding.get_device_error() != binding.RA_OK:
         raise RuntimeError("device error during the timed region")
     ms_step = ms / a.steps
