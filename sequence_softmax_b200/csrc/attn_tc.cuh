@@ -294,22 +294,28 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (T > 0) {
       const uint32_t tS[2] = {tmem + C::COL_S0, tmem + C::COL_S1};
       const uint32_t tO[2] = {tmem + C::COL_O0, tmem + C::COL_O1};
+      // Descriptors are built once; per k-step only the start-address field (the low 14
+      // bits, in 16-byte units) moves, by a constant. Addresses stay below 256 KB, so the
+      // add never carries into the neighbouring fields.
+      const uint32_t hi_sw128 = (1024u >> 4) | (1u << 14) | (2u << 29);  // SBO 1 KB, sm_100 version, 128B swizzle
+      const uint32_t lo_q[2] = {((sQ & 0x3FFFFu) >> 4) | (1u << 16),
+                                (((sQ + C::TILE_BYTES) & 0x3FFFFu) >> 4) | (1u << 16)};
+      const uint32_t lo_k = ((sKV & 0x3FFFFu) >> 4) | (1u << 16);                     // K-major, LBO 16 B
+      const uint32_t lo_v = ((sKV & 0x3FFFFu) >> 4) | ((uint32_t)(C::BOX_BYTES >> 4) << 16);  // MN-major, LBO one box
+      auto desc = [&](uint32_t lo) { return ((uint64_t)hi_sw128 << 32) | lo; };
       auto issue_s = [&](int t, int st) {
-        const uint32_t qa = sQ + t * C::TILE_BYTES;
-        const uint32_t ka = sKV + st * C::TILE_BYTES;
+        const uint32_t kb = lo_k + (uint32_t)st * (C::TILE_BYTES >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-          mma_bf16_ss(tS[t], sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), C::IDESC_S,
-                      kk > 0);
+          const uint32_t off = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
+          mma_bf16_ss(tS[t], desc(lo_q[t] + off), desc(kb + off), C::IDESC_S, kk > 0);
         }
       };
       auto issue_pv = [&](int t, int st, bool acc) {
-        const uint32_t va = sKV + st * C::TILE_BYTES;
+        const uint32_t vb = lo_v + (uint32_t)st * (C::TILE_BYTES >> 4);
 #pragma unroll
         for (int kk = 0; kk < TC_BN / 16; ++kk)
-          mma_bf16_ts(tO[t], tS[t] + kk * 8, sdesc_sw128(va + kk * 2048, C::BOX_BYTES, 1024), C::IDESC_PV,
-                      (acc || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tO[t], tS[t] + kk * 8, desc(vb + kk * (2048 >> 4)), C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
       };
       auto wait_all = [&](uint32_t bar, uint32_t parity) {
         return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
@@ -438,18 +444,17 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             for (int j = 0; j < TC_BN; ++j) sr[j] = (j <= lim) ? sr[j] : __float_as_uint(-INFINITY);
           }
 #define SV(j) __uint_as_float(sr[(j)])
-          float mx0 = fmax3(SV(0), SV(1), SV(2)), mx1 = fmax3(SV(3), SV(4), SV(5));
-          float mx2 = fmax3(SV(6), SV(7), SV(8)), mx3 = fmax3(SV(9), SV(10), SV(11));
+          float mxc[8];
 #pragma unroll
-          for (int j = 12; j < TC_BN - 8; j += 8) {
-            mx0 = fmax3(mx0, SV(j), SV(j + 1));
-            mx1 = fmax3(mx1, SV(j + 2), SV(j + 3));
-            mx2 = fmax3(mx2, SV(j + 4), SV(j + 5));
-            mx3 = fmax3(mx3, SV(j + 6), SV(j + 7));
+          for (int c = 0; c < 8; ++c) mxc[c] = fmax3(SV(2 * c), SV(2 * c + 1), SV(16 + 2 * c));
+#pragma unroll
+          for (int j = 32; j < TC_BN; j += 16) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) mxc[c] = fmax3(mxc[c], SV(j + 2 * c), SV(j + 2 * c + 1));
           }
-          mx0 = fmax3(mx0, SV(TC_BN - 4), SV(TC_BN - 3));
-          mx1 = fmax3(mx1, SV(TC_BN - 2), SV(TC_BN - 1));
-          const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) mxc[c] = fmaxf(mxc[c], SV(17 + 2 * c));
+          const float mx = fmaxf(fmax3(mxc[0], mxc[1], mxc[2]), fmax3(mxc[3], mxc[4], fmax3(mxc[5], mxc[6], mxc[7]))) * sl2;
           // Running max update (conditional rescale, see the file comment).
           float corr = 1.f;
           bool rescale = false;
