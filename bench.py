@@ -35,7 +35,7 @@ METRIC = "ring-attn fwd TFLOP/s (bf16, 1 B200), % of tensor peak; merge HBM GB/s
 PROFILE_JSON = os.path.join(ROOT, "profiles", "counters.json")
 KERNEL_SOURCES = {
     "attn_fwd_tc": ["sequence_softmax_b200/csrc/attn_tc.cuh", "sequence_softmax_b200/csrc/common.cuh"],
-    "merge": ["sequence_softmax_b200/csrc/merge.cuh", "sequence_softmax_b200/csrc/common.cuh"],
+    "merge": ["sequence_softmax_b200/csrc/merge.cuh"],
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "source": "fallback"}

@@ -128,6 +128,16 @@ const char* ra_status_string(ra_status status);
  */
 ra_status ra_get_device_error(cudaStream_t stream);
 
+/*
+ * ra_selftest_wait_timeout -- exercises the library's failure detection without faulting
+ * the GPU: launches one block whose thread waits on a shared-memory barrier that nothing
+ * signals, through the same bounded wait every kernel here uses. After limit_ns of device
+ * time (1 ms to 2 s) the wait gives up, records RA_ERR_TIMEOUT in the device error word and
+ * the kernel returns; the context stays usable. Read the outcome with
+ * ra_get_device_error(). Returns RA_ERR_INVALID_ARG for a limit outside the range.
+ */
+ra_status ra_selftest_wait_timeout(int64_t limit_ns, cudaStream_t stream);
+
 /* ABI version of this header (incremented on any signature change). */
 int ra_abi_version(void);
 

@@ -12,7 +12,7 @@ The binding module loads the shared library on first use and raises if it is mis
 """
 
 __all__ = ["partial", "merge", "ring_forward", "status_string", "get_device_error",
-           "library_path", "RaError"]
+           "selftest_wait_timeout", "library_path", "RaError"]
 
 
 def __getattr__(name):

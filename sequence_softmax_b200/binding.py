@@ -31,6 +31,7 @@ SIGNATURES = {
                                _i32, _vp, _vp, _vp]),
     "ra_status_string": (ctypes.c_char_p, [_i32]),
     "ra_get_device_error": (_i32, [_vp]),
+    "ra_selftest_wait_timeout": (_i32, [_i64, _vp]),
     "ra_abi_version": (_i32, []),
 }
 
@@ -94,6 +95,13 @@ def _dev(t: torch.Tensor, name: str):
 def get_device_error(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device error status code."""
     return load().ra_get_device_error(_stream_ptr(stream))
+
+
+def selftest_wait_timeout(limit_ns: int = 50_000_000, stream=None) -> int:
+    """Launch the failure-detection self-test (a bounded wait that must run out); returns the
+    device error status read afterwards (RA_ERR_TIMEOUT when detection works)."""
+    _check(load().ra_selftest_wait_timeout(int(limit_ns), _stream_ptr(stream)), "ra_selftest_wait_timeout")
+    return get_device_error(stream)
 
 
 def partial(q, k, v, causal: bool = False, scale: float | None = None,

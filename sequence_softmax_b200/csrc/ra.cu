@@ -12,6 +12,21 @@
 #define RA_ABI_VERSION 1
 
 namespace ra {
+
+// Failure-detection self-test: one thread waits on a barrier that nothing signals, through
+// the same bounded wait the attention kernel uses, and gives up after limit_ns.
+__global__ void selftest_wait_timeout_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, limit_ns);
+}
+
 namespace {
 
 // ---- cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda) ----
@@ -135,6 +150,12 @@ ra_status ra_get_device_error(cudaStream_t stream) {
   if (word & DEVERR_TIMEOUT) return RA_ERR_TIMEOUT;
   if (word & DEVERR_BOUNDS) return RA_ERR_DEVICE_BOUNDS;
   return RA_OK;
+}
+
+ra_status ra_selftest_wait_timeout(int64_t limit_ns, cudaStream_t stream) {
+  if (limit_ns < 1000000 || limit_ns > 2000000000) return RA_ERR_INVALID_ARG;
+  selftest_wait_timeout_kernel<<<1, 32, 0, stream>>>((uint64_t)limit_ns);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
 ra_status ra_partial(const void* q, const void* k, const void* v, ra_dtype dt, int B, int H, int64_t Lq,
