@@ -55,7 +55,7 @@ struct TcCfg {
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = 2 * TILE_BYTES;
   static constexpr int BAR_OFF = KV_OFF + NSTAGE * TILE_BYTES;
-  static constexpr int NBAR = 2 + 2 * NSTAGE + 2 + 2 + 2 + 1;
+  static constexpr int NBAR = 2 + 2 * NSTAGE + 2 + 2 + 2 + 1 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack to align the base to 1 KB
   static constexpr int COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
@@ -129,12 +129,13 @@ __device__ __forceinline__ void exp2_poly_pair(uint64_t x2, float& p0, float& p1
 }
 
 // P = exp2(s * sl2 - shift) for one row of 128 scores: writes P as bf16 pairs into TMEM
-// columns [0, 64) at tS and returns the row sums of the even and odd columns. With EMU,
+// columns [0, 64) at tS, arrives on bar_first_half once the first 32 columns (keys 0-63)
+// are stored, and returns the row sums of the even and odd columns. With EMU,
 // RA_EMU_PAIRS_OF_8 pairs in eight go through exp2_poly_pair (only on tiles without
 // masked scores).
 template <bool EMU>
 __device__ __forceinline__ void exp_tile(const uint32_t (&sr)[TC_BN], float sl2, float shift, uint32_t tS,
-                                         float& sum0, float& sum1) {
+                                         uint32_t bar_first_half, float& sum0, float& sum1) {
   const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-shift, -shift);
   uint64_t sum2a = f2_pack(0.f, 0.f), sum2b = sum2a;
 #pragma unroll
@@ -158,6 +159,13 @@ __device__ __forceinline__ void exp_tile(const uint32_t (&sr)[TC_BN], float sl2,
       pk[j] = pack_bf16x2(p0, p1);
     }
     RA_TMEM_ST32(tS + half * 32, pk);
+    if (half == 0) {
+      // P of keys 0-63 is complete: the MMA warp may start PV on it while the second
+      // half is computed.
+      tmem_wait_st();
+      tc_fence_before_sync();
+      mbar_arrive(bar_first_half);
+    }
   }
   float sa0, sa1, sb0, sb1;
   f2_unpack(sum2a, sa0, sa1);
@@ -184,6 +192,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   auto bar_p_full = [&](int t) { return bar0 + 8u * (4 + 2 * C::NSTAGE + t); };
   auto bar_o_done = [&](int t) { return bar0 + 8u * (6 + 2 * C::NSTAGE + t); };
   const uint32_t bar_drain = bar0 + 8u * (8 + 2 * C::NSTAGE);
+  auto bar_p_half = [&](int t) { return bar0 + 8u * (9 + 2 * C::NSTAGE + t); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
 
@@ -211,6 +220,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar_s_full(t), 1);
       mbar_init(bar_p_full(t), TC_BM);
+      mbar_init(bar_p_half(t), TC_BM);
       mbar_init(bar_o_done(t), 1);
     }
     mbar_init(bar_drain, 1);
@@ -311,14 +321,29 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           mma_bf16_ss(tS[t], desc(lo_q[t] + off), desc(kb + off), C::IDESC_S, kk > 0);
         }
       };
-      auto issue_pv = [&](int t, int st, bool acc) {
-        const uint32_t vb = lo_v + (uint32_t)st * (C::TILE_BYTES >> 4);
-#pragma unroll
-        for (int kk = 0; kk < TC_BN / 16; ++kk)
-          mma_bf16_ts(tO[t], tS[t] + kk * 8, desc(vb + kk * (2048 >> 4)), C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
-      };
       auto wait_all = [&](uint32_t bar, uint32_t parity) {
         return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+      };
+      // PV over keys 64h .. 64h + 63 (k-steps 4h .. 4h + 3).
+      auto issue_pv_half = [&](int t, int st, bool acc, int h) {
+        const uint32_t vb = lo_v + (uint32_t)st * (C::TILE_BYTES >> 4);
+#pragma unroll
+        for (int k4 = 0; k4 < TC_BN / 32; ++k4) {
+          const int kk = h * (TC_BN / 32) + k4;
+          mma_bf16_ts(tO[t], tS[t] + kk * 8, desc(vb + kk * (2048 >> 4)), C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      // PV of tile t: waits for each half of P separately.
+      auto pv_tile = [&](int t, int st, bool acc, uint32_t parity) {
+        if (!wait_all(bar_p_half(t), parity)) return false;
+        tc_fence_after_sync();
+        if (elect_one()) issue_pv_half(t, st, acc, 0);
+        __syncwarp();
+        if (!wait_all(bar_p_full(t), parity)) return false;
+        tc_fence_after_sync();
+        if (elect_one()) issue_pv_half(t, st, acc, 1);
+        __syncwarp();
+        return true;
       };
       bool ok = wait_all(bar_q_full(0), 0) && wait_all(bar_q_full(1), 0);
       // tile 0: K_0
@@ -340,10 +365,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const uint32_t pv = (uv / C::NSTAGE) & 1u, pk = (uk / C::NSTAGE) & 1u;
         const uint32_t pp = (uint32_t)(n - 1) & 1u;
         if (!(ok = wait_all(bar_kv_full(sv), pv))) break;
-        if (!(ok = wait_all(bar_p_full(0), pp))) break;
-        tc_fence_after_sync();
-        if (elect_one()) issue_pv(0, sv, n - 1 > 0);
-        __syncwarp();
+        if (!(ok = pv_tile(0, sv, n - 1 > 0, pp))) break;
         if (!(ok = wait_all(bar_kv_full(sk), pk))) break;
         tc_fence_after_sync();
         if (elect_one()) {
@@ -351,10 +373,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           tc_commit(bar_s_full(0));
         }
         __syncwarp();
-        if (!(ok = wait_all(bar_p_full(1), pp))) break;
-        tc_fence_after_sync();
+        if (!(ok = pv_tile(1, sv, n - 1 > 0, pp))) break;
         if (elect_one()) {
-          issue_pv(1, sv, n - 1 > 0);
           tc_commit(bar_kv_empty(sv));
           issue_s(1, sk);
           tc_commit(bar_s_full(1));
@@ -366,20 +386,14 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const uint32_t uv = 2u * (T - 1) + 1u;
         const int sv = uv % C::NSTAGE;
         const uint32_t pv = (uv / C::NSTAGE) & 1u, pp = (uint32_t)(T - 1) & 1u;
-        ok = wait_all(bar_kv_full(sv), pv) && wait_all(bar_p_full(0), pp);
+        ok = wait_all(bar_kv_full(sv), pv) && pv_tile(0, sv, T - 1 > 0, pp);
         if (ok) {
-          tc_fence_after_sync();
-          if (elect_one()) {
-            issue_pv(0, sv, T - 1 > 0);
-            tc_commit(bar_o_done(0));
-          }
+          if (elect_one()) tc_commit(bar_o_done(0));
           __syncwarp();
-          ok = wait_all(bar_p_full(1), pp);
+          ok = pv_tile(1, sv, T - 1 > 0, pp);
         }
         if (ok) {
-          tc_fence_after_sync();
           if (elect_one()) {
-            issue_pv(1, sv, T - 1 > 0);
             tc_commit(bar_o_done(1));
             tc_commit(bar_kv_empty(sv));
           }
@@ -481,9 +495,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           const float shift = (m == -INFINITY) ? 0.f : m;
           float sum0, sum1;
           if (full)
-            exp_tile<true>(sr, sl2, shift, tS, sum0, sum1);
+            exp_tile<true>(sr, sl2, shift, tS, bar_p_half(t), sum0, sum1);
           else
-            exp_tile<false>(sr, sl2, shift, tS, sum0, sum1);
+            exp_tile<false>(sr, sl2, shift, tS, bar_p_half(t), sum0, sum1);
 #undef SV
           l += sum0 + sum1;
           tmem_wait_st();
