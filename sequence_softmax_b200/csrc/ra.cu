@@ -195,17 +195,22 @@ ra_status ra_merge(const float* o_parts, const float* lse_parts, int n, int64_t 
   if (!o_parts || !lse_parts || !o_out || !aligned16(o_parts) || !aligned16(o_out)) return RA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(lse_parts) & 3u) || (lse_out && (reinterpret_cast<uintptr_t>(lse_out) & 3u)))
     return RA_ERR_INVALID_ARG;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t warps_needed = (rows + 1) / 2;
-  int64_t blocks = (warps_needed * 32 + MERGE_THREADS - 1) / MERGE_THREADS;
-  const int64_t cap = (int64_t)sms * 8;  // 8 resident blocks of 256 threads per SM
-  if (blocks > cap) blocks = cap;
-  if (out_dt == RA_BF16)
-    merge_kernel<true><<<(unsigned)blocks, MERGE_THREADS, 0, stream>>>(o_parts, lse_parts, n, rows, d, o_out, lse_out);
-  else
-    merge_kernel<false><<<(unsigned)blocks, MERGE_THREADS, 0, stream>>>(o_parts, lse_parts, n, rows, d, o_out, lse_out);
+  // One group of MERGE_LANES_PER_ROW lanes per row; the kernel is grid-stride beyond the cap.
+  int64_t blocks = (rows * MERGE_LANES_PER_ROW + MERGE_THREADS - 1) / MERGE_THREADS;
+  if (blocks > (1ll << 22)) blocks = 1ll << 22;
+  const unsigned g = (unsigned)blocks;
+  const bool bf = out_dt == RA_BF16;
+#define RA_MERGE_LAUNCH(CPL)                                                                             \
+  (bf ? merge_kernel<true, CPL><<<g, MERGE_THREADS, 0, stream>>>(o_parts, lse_parts, n, rows, d, o_out, lse_out) \
+      : merge_kernel<false, CPL><<<g, MERGE_THREADS, 0, stream>>>(o_parts, lse_parts, n, rows, d, o_out, lse_out))
+  switch (d) {
+    case 32: RA_MERGE_LAUNCH(1); break;
+    case 64: RA_MERGE_LAUNCH(2); break;
+    case 128: RA_MERGE_LAUNCH(4); break;
+    case 256: RA_MERGE_LAUNCH(8); break;
+    default: RA_MERGE_LAUNCH(0); break;
+  }
+#undef RA_MERGE_LAUNCH
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
