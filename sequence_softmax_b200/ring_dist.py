@@ -1,0 +1,165 @@
+"""Ring attention across GPUs: one process per GPU, K and V rotating around the ring.
+
+Each rank holds the query, key and value tokens of one virtual ring position (the
+contiguous, striped or zig-zag layout of ``include/ra.h``) and keeps its query block for the
+whole computation. At step s it receives the K and V of position (rank - s) mod W from its
+predecessor and forwards the block it holds to its successor ("Ring Attention 논문 분석",
+listing ``ring_attention_forward``; "Ring Attention" glossary, "How Ring Attention works").
+K and V travel as one message (lecture 013 notes: one large message instead of two small
+ones), posted before the step's compute so that the transfer overlaps it.
+
+Every arithmetic step runs in the library's kernels: ``ra_partial`` computes the partial
+state of the local queries against the block held (skipped when the block is wholly in the
+queries' future), and ``ra_merge`` folds it into the running (O, lse) state -- the lse
+associativity of the lecture 013 notes applied step by step. PyTorch provides memory,
+streams and the process group.
+
+The exchange uses the process group's point-to-point operations: with NCCL on CUDA tensors
+directly; with gloo (which only sends host tensors) through pinned host staging buffers.
+"""
+
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from . import binding
+
+
+def position_segments(layout: str, N: int, P: int, p: int):
+    """Token segments (tok0, stride, count) of virtual position p, in increasing token order."""
+    if layout == "contiguous":
+        if N % P:
+            raise ValueError("contiguous layout needs N divisible by P")
+        return [(p * (N // P), 1, N // P)]
+    if layout == "striped":
+        if N % P:
+            raise ValueError("striped layout needs N divisible by P")
+        return [(p, P, N // P)]
+    if layout == "zigzag":
+        if N % (2 * P):
+            raise ValueError("zig-zag layout needs N divisible by 2P")
+        c = N // (2 * P)
+        return [(p * c, 1, c), ((2 * P - 1 - p) * c, 1, c)]
+    raise ValueError(f"unknown layout {layout!r}")
+
+
+def segment_in_future(q_seg, k_seg) -> bool:
+    """True when every key token of k_seg is after every query token of q_seg (causal skip)."""
+    q0, qs, qn = q_seg
+    k0, ks, kn = k_seg
+    return kn == 0 or qn == 0 or k0 > q0 + qs * (qn - 1)
+
+
+def ring_schedule(rank: int, world: int):
+    """Positions whose K/V rank `rank` holds at steps 0..world-1: (rank - s) mod world."""
+    return [(rank - s) % world for s in range(world)]
+
+
+def _peers(rank: int, world: int):
+    return (rank + 1) % world, (rank - 1) % world
+
+
+class _Exchanger:
+    """Sends one tensor to the successor and receives the predecessor's into a second one."""
+
+    def __init__(self, group, like: torch.Tensor):
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+        self.send_to, self.recv_from = _peers(self.rank, self.world)
+        self.nccl = dist.get_backend(group) == "nccl"
+        if not self.nccl:
+            self.host_send = torch.empty(like.shape, dtype=like.dtype, pin_memory=like.is_cuda)
+            self.host_recv = torch.empty(like.shape, dtype=like.dtype, pin_memory=like.is_cuda)
+
+    def _gsend(self):
+        return dist.get_global_rank(self.group, self.send_to) if self.group is not None else self.send_to
+
+    def _grecv(self):
+        return dist.get_global_rank(self.group, self.recv_from) if self.group is not None else self.recv_from
+
+    def start(self, send: torch.Tensor, recv: torch.Tensor):
+        """Post the exchange; returns a handle for ``finish``."""
+        if self.nccl:
+            ops = [dist.P2POp(dist.isend, send, self._gsend(), self.group),
+                   dist.P2POp(dist.irecv, recv, self._grecv(), self.group)]
+            return dist.batch_isend_irecv(ops), recv
+        self.host_send.copy_(send)
+        # even ranks send first, odd ranks receive first: no cycle of blocking sends
+        if self.rank % 2 == 0:
+            reqs = [dist.isend(self.host_send, self._gsend(), self.group),
+                    dist.irecv(self.host_recv, self._grecv(), self.group)]
+        else:
+            reqs = [dist.irecv(self.host_recv, self._grecv(), self.group),
+                    dist.isend(self.host_send, self._gsend(), self.group)]
+        return reqs, recv
+
+    def finish(self, handle):
+        reqs, recv = handle
+        for r in reqs:
+            r.wait()
+        if not self.nccl:
+            recv.copy_(self.host_recv)
+        return recv
+
+
+def ring_forward_dist(q_local, k_local, v_local, N: int, layout: str = "contiguous", causal: bool = False,
+                      scale: float | None = None, group=None):
+    """Exact attention over a sequence of N tokens split across the ranks of `group`.
+
+    q_local, k_local, v_local: [B, H, N/W, d] CUDA tensors (bf16 with d in {64, 128}, or fp32)
+    holding the tokens of virtual position `rank` in increasing token order (for zig-zag,
+    chunk rank followed by chunk 2W-1-rank). Returns (O_local [B, H, N/W, d] in the input
+    dtype, lse_local [B, H, N/W] fp32) for the same tokens.
+    """
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    B, H, n_local, d = q_local.shape
+    segs = position_segments(layout, N, world, rank)
+    if sum(s[2] for s in segs) != n_local or k_local.shape != q_local.shape or v_local.shape != q_local.shape:
+        raise ValueError("local tensors must hold the N/W tokens of this rank's position")
+    scale = d ** -0.5 if scale is None else float(scale)
+
+    # Running state per query segment: parts[0] = running O (fp32), parts[1] = newest partial.
+    dev = q_local.device
+    q_segs, offs = [], 0
+    for seg in segs:
+        q_segs.append((q_local[:, :, offs:offs + seg[2]].contiguous(), seg, offs))
+        offs += seg[2]
+    state = []
+    for qs, seg, _ in q_segs:
+        rows = seg[2]
+        parts_o = torch.zeros(2, B, H, rows, d, device=dev, dtype=torch.float32)
+        parts_l = torch.full((2, B, H, rows), float("-inf"), device=dev, dtype=torch.float32)
+        state.append((parts_o, parts_l))
+
+    kv = torch.stack([k_local, v_local]).contiguous()     # one K||V message
+    kv_next = torch.empty_like(kv)
+    ex = _Exchanger(group, kv) if world > 1 else None
+    for s, src in enumerate(ring_schedule(rank, world)):
+        handle = ex.start(kv, kv_next) if (ex is not None and s < world - 1) else None
+        k_segs = position_segments(layout, N, world, src)
+        koff = 0
+        for kseg in k_segs:
+            kk = kv[0][:, :, koff:koff + kseg[2]].contiguous() if len(k_segs) > 1 else kv[0]
+            vv = kv[1][:, :, koff:koff + kseg[2]].contiguous() if len(k_segs) > 1 else kv[1]
+            koff += kseg[2]
+            for (qs, qseg, _), (parts_o, parts_l) in zip(q_segs, state):
+                if causal and segment_in_future(qseg, kseg):
+                    continue
+                binding.partial(qs, kk, vv, causal=causal, scale=scale, q_tok0=qseg[0], q_tok_stride=qseg[1],
+                                k_tok0=kseg[0], k_tok_stride=kseg[1], out=parts_o[1], lse=parts_l[1])
+                merged_o, merged_l = binding.merge(parts_o, parts_l, out_dtype=torch.float32)
+                parts_o[0].copy_(merged_o)
+                parts_l[0].copy_(merged_l)
+        if handle is not None:
+            kv_next = ex.finish(handle)
+            kv, kv_next = kv_next, kv
+
+    out = torch.empty_like(q_local)
+    lse = torch.empty(B, H, n_local, device=dev, dtype=torch.float32)
+    for (qs, seg, off), (parts_o, parts_l) in zip(q_segs, state):
+        out[:, :, off:off + seg[2]].copy_(parts_o[0])
+        lse[:, :, off:off + seg[2]].copy_(parts_l[0])
+    return out, lse

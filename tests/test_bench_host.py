@@ -29,7 +29,7 @@ def _rank_main(rank, world, port, out):
 
 def test_max_over_ranks_gloo_two_ranks():
     world = 2
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     port = 29500 + os.getpid() % 1000
     mp.spawn(_rank_main, args=(world, port, out), nprocs=world, join=True)
     assert out[0] == out[1] == 15.0
