@@ -20,9 +20,12 @@ Sources (cited by page title and section):
   (running max m, running sum l, running output o) and on causal imbalance
   (zig-zag placement).
 
+Backward (gradients of the same attention): ``oracle/backward.py``.
+
 Parity status of every function is stated in its module docstring.
 """
 
+from .backward import attention_backward, ring_backward  # noqa: F401
 from .ring import (  # noqa: F401
     NEG_INF,
     attention,
