@@ -1,5 +1,5 @@
 /*
- * ra.h -- C ABI of libra.so: the forward hot path of ring attention on one NVIDIA B200.
+ * ra.h -- C ABI of libra.so: ring attention (forward, merge and backward) on one NVIDIA B200.
  *
  * Ring attention computes exact softmax attention while a query block stays fixed and
  * key/value chunks arrive one at a time; each chunk's partial result is folded into a
@@ -117,6 +117,73 @@ ra_status ra_merge(const float* o_parts, const float* lse_parts, int n, int64_t 
 ra_status ra_ring_forward(const void* q, const void* k, const void* v, ra_dtype dt,
                           int B, int H, int64_t N, int d, float scale, int n_chunks, int causal,
                           ra_layout layout, void* o, float* lse, cudaStream_t stream);
+
+/*
+ * Backward pass ([BLOG] ring_attention_backward, with the causal mask the listing leaves
+ * out). With P = exp(S - lse) (S = q k^T * scale, lse from the forward) and upstream
+ * gradient dO of the output O:
+ *   dV = P^T dO,   dP = dO V^T,   D_i = sum_e dO_ie O_ie,
+ *   dS = P * (dP - D) * scale,   dQ = dS K,   dK = dS^T Q.
+ * In the ring, each position keeps Q, dO, O, lse and its dQ; the KV chunk travels with its
+ * dK, dV contributions, which are summed at the chunk's owner. The listing returns them
+ * with a reduce whose root differs per rank; that sum is the reading implemented here.
+ */
+
+/*
+ * ra_backward_delta -- the row term D_i = sum_e dO_ie O_ie (fp32 accumulation).
+ *   o, d_o     [rows, d]  dtype dt (O of the forward and its upstream gradient)
+ *   delta      [rows]     fp32, written
+ * Same dtype / d support as the forward. rows == 0 is a no-op.
+ */
+ra_status ra_backward_delta(const void* o, const void* d_o, ra_dtype dt, int64_t rows, int d,
+                            float* delta, cudaStream_t stream);
+
+/*
+ * ra_partial_backward -- one query block against one KV chunk: adds this pair's
+ * contributions to three fp32 accumulators (the caller zeroes them first):
+ *   dq_acc += dS K      [B, H, Lq, d] fp32
+ *   dk_acc += dS^T Q    [B, H, Lk, d] fp32
+ *   dv_acc += P^T dO    [B, H, Lk, d] fp32
+ *   q, d_o     [B, H, Lq, d]  dtype dt
+ *   k, v       [B, H, Lk, d]  dtype dt
+ *   lse        [B, H, Lq]     fp32, the FINAL log-sum-exp of each query row (over all keys,
+ *                             e.g. from ra_ring_forward or ra_merge), so that P is the true
+ *                             softmax probability
+ *   delta      [B, H, Lq]     fp32, from ra_backward_delta on the final O
+ *   causal and the token arguments as in ra_partial.
+ * The bf16 kernel adds dq_acc with atomic vector adds (the order of the additions, and so
+ * the last bits of dq_acc, may differ between runs); dk_acc and dv_acc are read, added to
+ * and written by the one CTA that owns each key row. Lq == 0 or Lk == 0 is a no-op.
+ */
+ra_status ra_partial_backward(const void* q, const void* k, const void* v, const void* d_o,
+                              const float* lse, const float* delta, ra_dtype dt,
+                              int B, int H, int64_t Lq, int64_t Lk, int d, float scale, int causal,
+                              int64_t q_tok0, int64_t q_tok_stride, int64_t k_tok0, int64_t k_tok_stride,
+                              float* dq_acc, float* dk_acc, float* dv_acc, cudaStream_t stream);
+
+/*
+ * ra_ring_backward_workspace_bytes -- bytes of the caller-owned workspace ra_ring_backward
+ * needs: B*H*N*(d+1)*4 for bf16 (an fp32 dQ accumulator and D), B*H*N*4 for fp32 (D).
+ * Returns -1 for negative sizes.
+ */
+int64_t ra_ring_backward_workspace_bytes(ra_dtype dt, int B, int H, int64_t N, int d);
+
+/*
+ * ra_ring_backward -- gradients of ra_ring_forward's output, by the ring: KV chunk c meets
+ * the query positions c, c+1, ... (mod P) in turn; each key tile's dK, dV accumulate on chip
+ * and are written once, dQ is accumulated in fp32. Three launches on `stream`: D (and a
+ * zeroed dQ accumulator), the gradient kernel(s), and for bf16 the dQ conversion.
+ *   q, k, v, o, d_o  [B, H, N, d]  dtype dt, natural token order
+ *   lse              [B, H, N]     fp32 (from ra_ring_forward)
+ *   dq, dk, dv       [B, H, N, d]  dtype dt, written
+ *   workspace        device memory of at least ra_ring_backward_workspace_bytes() bytes,
+ *                    16-byte aligned, owned by the caller; its contents are scratch
+ * Shape rules as ra_ring_forward. RA_ERR_INVALID_ARG if workspace_bytes is too small.
+ */
+ra_status ra_ring_backward(const void* q, const void* k, const void* v, const void* o, const void* d_o,
+                           const float* lse, ra_dtype dt, int B, int H, int64_t N, int d, float scale,
+                           int n_chunks, int causal, ra_layout layout, void* dq, void* dk, void* dv,
+                           void* workspace, int64_t workspace_bytes, cudaStream_t stream);
 
 /* Static, human-readable name of a status code (never NULL). */
 const char* ra_status_string(ra_status status);

@@ -25,7 +25,7 @@ Backward (gradients of the same attention): ``oracle/backward.py``.
 Parity status of every function is stated in its module docstring.
 """
 
-from .backward import attention_backward, ring_backward  # noqa: F401
+from .backward import attention_backward, backward_rows, delta, partial_backward, ring_backward  # noqa: F401
 from .ring import (  # noqa: F401
     NEG_INF,
     attention,

@@ -29,6 +29,12 @@ SIGNATURES = {
     "ra_merge": (_i32, [_vp, _vp, _i32, _i64, _i32, _vp, _i32, _vp, _vp]),
     "ra_ring_forward": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i64, _i32, _f32, _i32, _i32,
                                _i32, _vp, _vp, _vp]),
+    "ra_backward_delta": (_i32, [_vp, _vp, _i32, _i64, _i32, _vp, _vp]),
+    "ra_partial_backward": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i64, _i64, _i32, _f32, _i32,
+                                   _i64, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "ra_ring_backward_workspace_bytes": (_i64, [_i32, _i32, _i32, _i64, _i32]),
+    "ra_ring_backward": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i64, _i32, _f32, _i32, _i32,
+                                _i32, _vp, _vp, _vp, _vp, _i64, _vp]),
     "ra_status_string": (ctypes.c_char_p, [_i32]),
     "ra_get_device_error": (_i32, [_vp]),
     "ra_selftest_wait_timeout": (_i32, [_i64, _vp]),
@@ -192,3 +198,88 @@ def ring_forward(q, k, v, n_chunks: int, causal: bool = False, layout: str = "co
                                 lse.data_ptr() if return_lse else None, _stream_ptr(stream))
     _check(st, "ra_ring_forward")
     return out, (lse if return_lse else None)
+
+
+def backward_delta(o, d_o, out=None, stream=None):
+    """D = rowsum(dO * O) -> fp32 [...] for o, d_o [..., d]."""
+    _dev(o, "o")
+    _dev(d_o, "d_o")
+    if d_o.shape != o.shape or d_o.dtype != o.dtype:
+        raise ValueError("o and d_o must share shape and dtype")
+    d = o.shape[-1]
+    rows = o.numel() // d if d else 0
+    out = torch.empty(o.shape[:-1], device=o.device, dtype=torch.float32) if out is None else out
+    _dev(out, "out")
+    st = load().ra_backward_delta(o.data_ptr(), d_o.data_ptr(), _dtype_code(o), rows, d, out.data_ptr(),
+                                  _stream_ptr(stream))
+    _check(st, "ra_backward_delta")
+    return out
+
+
+def partial_backward(q, k, v, d_o, lse, delta, dq_acc, dk_acc, dv_acc, causal: bool = False,
+                     scale: float | None = None, q_tok0: int = 0, q_tok_stride: int = 1, k_tok0: int = 0,
+                     k_tok_stride: int = 1, stream=None):
+    """Adds one (query block, KV chunk) pair's gradients to fp32 accumulators (in place).
+
+    q, d_o [B,H,Lq,d]; k, v [B,H,Lk,d]; lse, delta [B,H,Lq] fp32 (final lse of the forward and
+    D = rowsum(dO * O)); dq_acc [B,H,Lq,d], dk_acc / dv_acc [B,H,Lk,d] fp32.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (d_o, "d_o"), (lse, "lse"), (delta, "delta"),
+                 (dq_acc, "dq_acc"), (dk_acc, "dk_acc"), (dv_acc, "dv_acc")):
+        _dev(t, n)
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    if k.shape != (B, H, Lk, d) or v.shape != k.shape or d_o.shape != q.shape:
+        raise ValueError("k, v must be [B, H, Lk, d] and d_o [B, H, Lq, d]")
+    if any(t.dtype != q.dtype for t in (k, v, d_o)):
+        raise ValueError("q, k, v, d_o must share a dtype")
+    if any(t.dtype != torch.float32 for t in (lse, delta, dq_acc, dk_acc, dv_acc)):
+        raise TypeError("lse, delta and the accumulators are float32")
+    if dq_acc.shape != q.shape or dk_acc.shape != k.shape or dv_acc.shape != k.shape:
+        raise ValueError("accumulators must match q / k shapes")
+    scale = d ** -0.5 if scale is None else float(scale)
+    st = load().ra_partial_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), d_o.data_ptr(), lse.data_ptr(),
+                                    delta.data_ptr(), _dtype_code(q), B, H, Lq, Lk, d, scale, int(bool(causal)),
+                                    q_tok0, q_tok_stride, k_tok0, k_tok_stride, dq_acc.data_ptr(),
+                                    dk_acc.data_ptr(), dv_acc.data_ptr(), _stream_ptr(stream))
+    _check(st, "ra_partial_backward")
+    return dq_acc, dk_acc, dv_acc
+
+
+def ring_backward_workspace_bytes(dtype, B: int, H: int, N: int, d: int) -> int:
+    code = RA_BF16 if dtype == torch.bfloat16 else RA_F32
+    return int(load().ra_ring_backward_workspace_bytes(code, B, H, N, d))
+
+
+def ring_backward(q, k, v, o, d_o, lse, n_chunks: int, causal: bool = False, layout: str = "contiguous",
+                  scale: float | None = None, workspace=None, out=None, stream=None):
+    """Gradients (dQ, dK, dV) of ``ring_forward``'s output for upstream gradient d_o.
+
+    q, k, v, o, d_o [B,H,N,d] in one dtype, lse [B,H,N] fp32 from ring_forward. ``workspace``
+    (a uint8 CUDA tensor of at least ring_backward_workspace_bytes bytes) is allocated when
+    not given; ``out`` may be a (dq, dk, dv) tuple of preallocated tensors.
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (d_o, "d_o"), (lse, "lse")):
+        _dev(t, n)
+    B, H, N, d = q.shape
+    if any(t.shape != q.shape or t.dtype != q.dtype for t in (k, v, o, d_o)):
+        raise ValueError("q, k, v, o, d_o must share shape [B, H, N, d] and dtype")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N):
+        raise ValueError("lse must be float32 [B, H, N]")
+    if layout not in LAYOUTS:
+        raise ValueError(f"layout must be one of {sorted(LAYOUTS)}")
+    scale = d ** -0.5 if scale is None else float(scale)
+    need = ring_backward_workspace_bytes(q.dtype, B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
+    _dev(workspace, "workspace")
+    dq, dk, dv = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)) if out is None else out
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _dev(t, n)
+    st = load().ra_ring_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), d_o.data_ptr(),
+                                 lse.data_ptr(), _dtype_code(q), B, H, N, d, scale, int(n_chunks),
+                                 int(bool(causal)), LAYOUTS[layout], dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                 workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                 _stream_ptr(stream))
+    _check(st, "ra_ring_backward")
+    return dq, dk, dv

@@ -1,0 +1,353 @@
+// bwd.cuh -- backward pass of ring attention: the problem plan, the key-tile / query-tile
+// walk, the row term D, the fp32 -> bf16 conversion of the dQ accumulator and the fp32
+// CUDA-core backward kernels.
+//
+// Gradients of O = softmax(S) V with S = Q K^T * scale ([BLOG] ring_attention_backward):
+//   P = exp(S - lse)            recomputed from the forward's log-sum-exp, no max pass
+//   dV = P^T dO                 dP = dO V^T
+//   D_i = sum_e dO_ie O_ie      (= sum_j P_ij dP_ij)
+//   dS = P * (dP - D) * scale   dQ = dS K      dK = dS^T Q
+// with the causal mask of the forward (key token j visible to query token i iff j <= i),
+// which that listing leaves out. In the ring, position p keeps Q_p, dO_p, O_p and lse_p;
+// at step s it receives KV chunk (p - s) mod P, adds dS K to its own dQ_p and hands the
+// chunk's dK, dV contributions back to the chunk's owner, where they are summed (the
+// listing's reduce to a per-rank root is read as that sum). Equivalently, KV chunk c meets
+// the query positions c, c + 1, ... (mod P) in turn: that is the order the kernels here walk.
+#pragma once
+
+#include "common.cuh"
+#include "attn_simt.cuh"
+
+namespace ra {
+
+struct BwdPlan {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* d_o;
+  const float* lse;     // [BH, q_rows] natural-log lse of the forward
+  const float* delta;   // [BH, q_rows] D = rowsum(dO * O)
+  float* dq;            // [BH, q_rows, d] fp32 (accumulated with atomics by the tensor-core kernel)
+  void* dk;             // [BH, k_rows, d]
+  void* dv;             // [BH, k_rows, d]
+  int BH;
+  int d;
+  int P;
+  int layout;
+  int causal;
+  int accumulate;       // 1: dq, dk, dv are fp32 accumulators (+=); 0: written
+  int dkdv_bf16;        // 1: dk, dv written as bf16 (tensor-core kernel, accumulate == 0)
+  int64_t q_rows, k_rows, q_seg_len, k_seg_len;
+  int64_t q_tok0, q_tok_stride, k_tok0, k_tok_stride;
+  float scale;
+  float scale_log2;
+};
+
+constexpr int BWD_TILE = 128;  // keys per key tile and query rows per query tile
+
+// The key tile a CTA owns: tile j0 / 128 of segment `seg` of position c.
+struct KTile {
+  int c;
+  Seg seg;
+  int64_t j0;
+};
+
+// Units within one head, earliest tokens first: under the causal mask the earliest keys are
+// seen by the most queries, so the longest-running CTAs start first.
+__device__ __forceinline__ KTile decode_ktile(const BwdPlan& pl, int unit) {
+  KTile t;
+  const int P = pl.P;
+  const int64_t nkt = (pl.k_seg_len + BWD_TILE - 1) / BWD_TILE;
+  int si = 0;
+  int64_t jt;
+  if (pl.layout == RA_LAYOUT_STRIPED) {
+    jt = unit / P;
+    t.c = unit % P;
+  } else if (pl.layout == RA_LAYOUT_ZIGZAG) {
+    const int gc = (int)(unit / nkt);  // global chunk
+    jt = unit % nkt;
+    if (gc < P) { t.c = gc; si = 0; } else { t.c = 2 * P - 1 - gc; si = 1; }
+  } else {
+    t.c = (int)(unit / nkt);
+    jt = unit % nkt;
+  }
+  t.seg = segment_of(pl.layout, P, pl.k_seg_len, t.c, si);
+  t.j0 = jt * BWD_TILE;
+  return t;
+}
+
+__device__ __forceinline__ int64_t ktile_token_min(const BwdPlan& pl, const KTile& kt) {
+  return pl.k_tok0 + pl.k_tok_stride * (kt.seg.row0 + kt.seg.stride * kt.j0);
+}
+
+// First local row of query segment qs that sees a key of token >= tk_min (causal), else 0.
+__host__ __device__ __forceinline__ int64_t first_seeing_row(const BwdPlan& pl, const Seg& qs, int64_t tk_min) {
+  if (!pl.causal) return 0;
+  const int64_t tq0 = pl.q_tok0 + pl.q_tok_stride * qs.row0;
+  const int64_t tqs = pl.q_tok_stride * qs.stride;
+  if (tk_min <= tq0) return 0;
+  return (tk_min - tq0 + tqs - 1) / tqs;
+}
+
+// Calls f(qs, i0) for every 128-row query tile (local rows i0 .. i0 + 127 of segment qs)
+// that can see a key of the tile, in ring order: positions c, c + 1, ... (mod P).
+// Stops when f returns false.
+template <class F>
+__device__ __forceinline__ void walk_q_tiles(const BwdPlan& pl, const KTile& kt, F&& f) {
+  const int64_t tk_min = ktile_token_min(pl, kt);
+  const int nqs = num_segments(pl.layout);
+  for (int s = 0; s < pl.P; ++s) {
+    int p = kt.c + s;
+    if (p >= pl.P) p -= pl.P;
+    for (int si = 0; si < nqs; ++si) {
+      const Seg qs = segment_of(pl.layout, pl.P, pl.q_seg_len, p, si);
+      const int64_t first = first_seeing_row(pl, qs, tk_min);
+      if (first >= qs.count) continue;
+      const int64_t ntile = (qs.count + BWD_TILE - 1) / BWD_TILE;
+      for (int64_t qt = first / BWD_TILE; qt < ntile; ++qt)
+        if (!f(qs, qt * BWD_TILE)) return;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// D_i = sum_e dO_ie O_ie, one group of 8 lanes per row; optionally zeroes row i of an fp32
+// [rows, d] accumulator in the same pass.
+// ------------------------------------------------------------------------------------
+constexpr int DELTA_THREADS = 256;
+
+template <bool BF16>
+__global__ void __launch_bounds__(DELTA_THREADS)
+bwd_delta_kernel(const void* __restrict__ o, const void* __restrict__ d_o, int64_t rows, int d,
+                 float* __restrict__ delta, float* __restrict__ zero_rows) {
+  const int g = threadIdx.x & 7;
+  const int64_t groups = (int64_t)gridDim.x * (DELTA_THREADS / 8);
+  for (int64_t r = (int64_t)blockIdx.x * (DELTA_THREADS / 8) + (threadIdx.x >> 3); r < rows; r += groups) {
+    float acc = 0.f;
+    if (BF16) {
+      // d is a multiple of 8: 16-byte chunks of 8 bf16
+      const uint4* a = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(o) + r * d);
+      const uint4* b = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(d_o) + r * d);
+      for (int c = g; c < d / 8; c += 8) {
+        const uint4 x = __ldcs(a + c), y = __ldcs(b + c);
+        const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xs[t]));
+          const float2 yf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ys[t]));
+          acc = fmaf(xf.x, yf.x, acc);
+          acc = fmaf(xf.y, yf.y, acc);
+        }
+      }
+    } else {
+      const float* a = static_cast<const float*>(o) + r * d;
+      const float* b = static_cast<const float*>(d_o) + r * d;
+      for (int e = g; e < d; e += 8) acc = fmaf(a[e], b[e], acc);
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+    if (g == 0) delta[r] = acc;
+    if (zero_rows != nullptr) {
+      float4* z = reinterpret_cast<float4*>(zero_rows + r * d);  // d % 4 == 0 here
+      for (int c = g; c < d / 4; c += 8) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+}
+
+// out[i] = bf16(acc[i]), n a multiple of 4.
+__global__ void __launch_bounds__(256)
+f32_to_bf16_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ out, int64_t n4) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 x = __ldcs(reinterpret_cast<const float4*>(acc) + i);
+    uint2 w;
+    w.x = pack_bf16x2(x.x, x.y);
+    w.y = pack_bf16x2(x.z, x.w);
+    reinterpret_cast<uint2*>(out)[i] = w;
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// fp32 backward on the CUDA cores (the fp32 path must match the definition within 1e-5,
+// which rules out tf32 tensor cores). Two kernels, no atomics:
+//   dkdv: one warp per key row, walking the query rows that see it in ring order;
+//         lane l scores query row i0 + l (full-d dot products), then the warp
+//         accumulates dV_j += P_ij dO_i and dK_j += dS_ij Q_i over those 32 rows.
+//   dq:   one warp per query row, walking the visible keys in the forward's ring order.
+// ------------------------------------------------------------------------------------
+__device__ __forceinline__ float bwd_prob(float s_scaled, float lse) {
+  return lse == -INFINITY ? 0.f : expf(s_scaled - lse);
+}
+
+// grid: x = ceil(key rows per position / SIMT_WARPS), y = P, z = B*H.
+__global__ void __launch_bounds__(SIMT_WARPS * 32)
+bwd_dkdv_simt_f32_kernel(const BwdPlan pl, int64_t rows_per_pos) {
+  __shared__ float sk[SIMT_WARPS][SIMT_DMAX];
+  __shared__ float sv[SIMT_WARPS][SIMT_DMAX];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t lj = (int64_t)blockIdx.x * SIMT_WARPS + warp;
+  const int c = blockIdx.y;
+  const int bh = blockIdx.z;
+  if (lj >= rows_per_pos) return;
+  const int d = pl.d;
+  const int sk_i = (int)(lj / pl.k_seg_len);
+  const Seg ks = segment_of(pl.layout, pl.P, pl.k_seg_len, c, sk_i);
+  const int64_t krow = ks.row0 + ks.stride * (lj - (int64_t)sk_i * pl.k_seg_len);
+  const int64_t tk = pl.k_tok0 + pl.k_tok_stride * krow;
+  const float* kp = static_cast<const float*>(pl.k) + ((int64_t)bh * pl.k_rows + krow) * d;
+  const float* vp = static_cast<const float*>(pl.v) + ((int64_t)bh * pl.k_rows + krow) * d;
+  for (int e = lane; e < d; e += 32) {
+    sk[warp][e] = kp[e];
+    sv[warp][e] = vp[e];
+  }
+  __syncwarp();
+  const float* qb = static_cast<const float*>(pl.q) + (int64_t)bh * pl.q_rows * d;
+  const float* ob = static_cast<const float*>(pl.d_o) + (int64_t)bh * pl.q_rows * d;
+  const float* lb = pl.lse + (int64_t)bh * pl.q_rows;
+  const float* db = pl.delta + (int64_t)bh * pl.q_rows;
+  float dk[SIMT_DMAX / 32], dv[SIMT_DMAX / 32];
+#pragma unroll
+  for (int t = 0; t < SIMT_DMAX / 32; ++t) dk[t] = dv[t] = 0.f;
+
+  const int nqs = num_segments(pl.layout);
+  for (int s = 0; s < pl.P; ++s) {
+    int p = c + s;
+    if (p >= pl.P) p -= pl.P;
+    for (int si = 0; si < nqs; ++si) {
+      const Seg qs = segment_of(pl.layout, pl.P, pl.q_seg_len, p, si);
+      for (int64_t i0 = first_seeing_row(pl, qs, tk); i0 < qs.count; i0 += 32) {
+        const int64_t i = i0 + lane;
+        const int64_t qrow = qs.row0 + qs.stride * i;
+        float pij = 0.f, dsij = 0.f;
+        if (i < qs.count && (!pl.causal || tk <= pl.q_tok0 + pl.q_tok_stride * qrow)) {
+          const float* qp = qb + qrow * d;
+          const float* op = ob + qrow * d;
+          float dot = 0.f, dpd = 0.f;
+          for (int e = 0; e < d; ++e) {
+            dot = fmaf(qp[e], sk[warp][e], dot);
+            dpd = fmaf(op[e], sv[warp][e], dpd);
+          }
+          pij = bwd_prob(dot * pl.scale, lb[qrow]);
+          dsij = pij * (dpd - db[qrow]) * pl.scale;
+        }
+        const int64_t nj = min((int64_t)32, qs.count - i0);
+        for (int jj = 0; jj < nj; ++jj) {
+          const float pb = __shfl_sync(0xffffffffu, pij, jj);
+          const float db2 = __shfl_sync(0xffffffffu, dsij, jj);
+          if (pb == 0.f && db2 == 0.f) continue;  // uniform across the warp
+          const int64_t r = qs.row0 + qs.stride * (i0 + jj);
+          const float* qp = qb + r * d;
+          const float* op = ob + r * d;
+#pragma unroll
+          for (int t = 0; t < SIMT_DMAX / 32; ++t) {
+            const int e = lane + 32 * t;
+            if (e < d) {
+              dv[t] = fmaf(pb, op[e], dv[t]);
+              dk[t] = fmaf(db2, qp[e], dk[t]);
+            }
+          }
+        }
+      }
+    }
+  }
+  float* dkp = static_cast<float*>(pl.dk) + ((int64_t)bh * pl.k_rows + krow) * d;
+  float* dvp = static_cast<float*>(pl.dv) + ((int64_t)bh * pl.k_rows + krow) * d;
+#pragma unroll
+  for (int t = 0; t < SIMT_DMAX / 32; ++t) {
+    const int e = lane + 32 * t;
+    if (e < d) {
+      if (pl.accumulate) {
+        dkp[e] += dk[t];
+        dvp[e] += dv[t];
+      } else {
+        dkp[e] = dk[t];
+        dvp[e] = dv[t];
+      }
+    }
+  }
+}
+
+// grid: x = ceil(query rows per position / SIMT_WARPS), y = P, z = B*H.
+__global__ void __launch_bounds__(SIMT_WARPS * 32)
+bwd_dq_simt_f32_kernel(const BwdPlan pl, int64_t rows_per_pos) {
+  __shared__ float sq[SIMT_WARPS][SIMT_DMAX];
+  __shared__ float so[SIMT_WARPS][SIMT_DMAX];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t li = (int64_t)blockIdx.x * SIMT_WARPS + warp;
+  const int p = blockIdx.y;
+  const int bh = blockIdx.z;
+  if (li >= rows_per_pos) return;
+  const int d = pl.d;
+  const int si = (int)(li / pl.q_seg_len);
+  const Seg qs = segment_of(pl.layout, pl.P, pl.q_seg_len, p, si);
+  const int64_t qrow = qs.row0 + qs.stride * (li - (int64_t)si * pl.q_seg_len);
+  const int64_t tq = pl.q_tok0 + pl.q_tok_stride * qrow;
+  const float* qp = static_cast<const float*>(pl.q) + ((int64_t)bh * pl.q_rows + qrow) * d;
+  const float* op = static_cast<const float*>(pl.d_o) + ((int64_t)bh * pl.q_rows + qrow) * d;
+  for (int e = lane; e < d; e += 32) {
+    sq[warp][e] = qp[e];
+    so[warp][e] = op[e];
+  }
+  __syncwarp();
+  const float lse = pl.lse[(int64_t)bh * pl.q_rows + qrow];
+  const float Di = pl.delta[(int64_t)bh * pl.q_rows + qrow];
+  const float* kb = static_cast<const float*>(pl.k) + (int64_t)bh * pl.k_rows * d;
+  const float* vb = static_cast<const float*>(pl.v) + (int64_t)bh * pl.k_rows * d;
+  float dq[SIMT_DMAX / 32];
+#pragma unroll
+  for (int t = 0; t < SIMT_DMAX / 32; ++t) dq[t] = 0.f;
+
+  // The key-side visibility test of the forward (keys of token <= tq), on the key plan.
+  Plan kp{};
+  kp.causal = pl.causal;
+  kp.k_tok0 = pl.k_tok0;
+  kp.k_tok_stride = pl.k_tok_stride;
+  const int nks = num_segments(pl.layout);
+  for (int s = 0; s < pl.P; ++s) {
+    int c = p - s;
+    if (c < 0) c += pl.P;
+    for (int sk_i = 0; sk_i < nks; ++sk_i) {
+      const Seg ks = segment_of(pl.layout, pl.P, pl.k_seg_len, c, sk_i);
+      const int64_t nvis = visible_prefix(kp, ks, tq);
+      for (int64_t j0 = 0; j0 < nvis; j0 += 32) {
+        const int64_t j = j0 + lane;
+        const int64_t krow = ks.row0 + ks.stride * j;
+        float dsij = 0.f;
+        if (j < nvis && (!pl.causal || pl.k_tok0 + pl.k_tok_stride * krow <= tq)) {
+          const float* kr = kb + krow * d;
+          const float* vr = vb + krow * d;
+          float dot = 0.f, dpd = 0.f;
+          for (int e = 0; e < d; ++e) {
+            dot = fmaf(sq[warp][e], kr[e], dot);
+            dpd = fmaf(so[warp][e], vr[e], dpd);
+          }
+          dsij = bwd_prob(dot * pl.scale, lse) * (dpd - Di) * pl.scale;
+        }
+        const int64_t nj = min((int64_t)32, nvis - j0);
+        for (int jj = 0; jj < nj; ++jj) {
+          const float db2 = __shfl_sync(0xffffffffu, dsij, jj);
+          if (db2 == 0.f) continue;
+          const float* kr = kb + (ks.row0 + ks.stride * (j0 + jj)) * d;
+#pragma unroll
+          for (int t = 0; t < SIMT_DMAX / 32; ++t) {
+            const int e = lane + 32 * t;
+            if (e < d) dq[t] = fmaf(db2, kr[e], dq[t]);
+          }
+        }
+      }
+    }
+  }
+  float* dqp = pl.dq + ((int64_t)bh * pl.q_rows + qrow) * d;
+#pragma unroll
+  for (int t = 0; t < SIMT_DMAX / 32; ++t) {
+    const int e = lane + 32 * t;
+    if (e < d) {
+      if (pl.accumulate) dqp[e] += dq[t];
+      else dqp[e] = dq[t];
+    }
+  }
+}
+
+}  // namespace ra

@@ -1,0 +1,450 @@
+// bwd_tc.cuh -- bf16 ring-attention backward on the 5th-generation tensor cores (sm_100a).
+//
+// Key-stationary: one CTA owns a tile of 128 keys of one virtual ring position and walks
+// every 128-row query tile that can see it, in ring order (positions c, c + 1, ... as the
+// KV chunk travels; see bwd.cuh). Its dK and dV stay in tensor memory for the whole walk
+// and are written once at the end, which is the "sum at the chunk's owner" of the ring
+// backward; dQ of each query tile is added to an fp32 accumulator in global memory.
+//
+// Per query tile i (Q_i, dO_i, lse_i, D_i staged by TMA / the producer warp):
+//   S^T  = K Q_i^T             (M = keys, N = queries, K = d; both operands K-major)
+//   dP^T = V dO_i^T            (same form)
+//   P^T  = exp2(S^T scale log2e - lse_i log2e), masked; bf16 into the S columns of TMEM
+//   dV  += P^T dO_i            (A = P^T from TMEM, B = dO_i MN-major)
+//   dS^T = P^T (dP^T - D_i) scale, bf16 into a 128B-swizzled shared-memory tile
+//   dK  += dS^T Q_i            (A = dS^T K-major, B = Q_i MN-major)
+//   dQ_i = dS K                (A = the same dS tile read MN-major, B = K MN-major)
+// so each (query tile, key tile) pair costs five 128 x 128 x d GEMMs and one exponential per
+// score, and P and dS never leave the SM.
+//
+// Warp roles (384 threads, 3 warpgroups; setmaxnreg moves registers to the math warps):
+//   warps 0-3, 4-7  math: thread t of warpgroup g owns key row t (TMEM lane t) and query
+//                   columns 64g .. 64g + 63 of S^T / dP^T; for dQ it owns query row t and
+//                   columns g d/2 .. g d/2 + d/2 - 1
+//   warp 8          producer: K and V once, then Q_i and dO_i by TMA into a 2-stage ring,
+//                   with lse_i log2e and D_i stored beside them
+//   warp 9          MMA issuer (the whole warp loops, one elected lane issues)
+//
+// Tensor memory (512 columns): S^T/P^T [0,128) | dP^T [128,256) | dV | dK, with dQ_i in the
+// dP^T columns for d = 128 (issued after the math warps have read dP^T; the next dP^T waits
+// until dQ_i has been read) and in free columns [256, 320) for d = 64.
+//
+// Query rows beyond a segment's end get lse log2e = +inf and D = 0, so their P and dS are
+// exactly 0 and they add nothing to dK, dV; key rows beyond the end get P = dS = 0 and are
+// not written. A query row whose forward lse is -inf saw no key and gets P = 0 as well.
+#pragma once
+
+#include "bwd.cuh"
+
+namespace ra {
+
+constexpr int BW_THREADS = 384;
+constexpr int BW_WARP_PRODUCER = 8;
+constexpr int BW_WARP_MMA = 9;
+constexpr int BW_REGS_MATH = 216;   // 2 x 216 + 72 = 504 = 168 * 384 / 128
+constexpr int BW_REGS_OTHER = 72;
+constexpr int BW_NSTAGE = 2;
+constexpr int BW_TMEM_COLS = 512;
+
+template <int D>
+struct BwCfg {
+  static_assert(D == 64 || D == 128, "head dimension 64 or 128");
+  static constexpr int BOX_BYTES = BWD_TILE * 64 * 2;       // one TMA box: 128 rows x 64 bf16
+  static constexpr int NBOX = D / 64;
+  static constexpr int TILE_BYTES = NBOX * BOX_BYTES;       // a K, V, Q or dO tile
+  static constexpr int DS_BYTES = 2 * BOX_BYTES;            // dS^T: 128 keys x 128 queries
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = TILE_BYTES;
+  static constexpr int Q_OFF = 2 * TILE_BYTES;              // stage s: Q at +2s TILE, dO at +(2s+1) TILE
+  static constexpr int DS_OFF = Q_OFF + BW_NSTAGE * 2 * TILE_BYTES;
+  static constexpr int LD_OFF = DS_OFF + DS_BYTES;          // stage s: lse log2e [128], D [128]
+  static constexpr int BAR_OFF = LD_OFF + BW_NSTAGE * 2 * BWD_TILE * 4;
+  static constexpr int NBAR = 16;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16;
+  static constexpr int COL_S = 0, COL_DP = 128;
+  static constexpr int COL_DQ = (D == 128) ? 128 : 256;
+  static constexpr int COL_DV = (D == 128) ? 256 : 320;
+  static constexpr int COL_DK = COL_DV + D;
+  static constexpr bool DQ_IN_DP = D == 128;
+  static constexpr uint32_t IDESC_SS = idesc_bf16_f32_ab(128, 128, false, false);
+  static constexpr uint32_t IDESC_KMN = idesc_bf16_f32_ab(128, D, false, true);  // dV, dK
+  static constexpr uint32_t IDESC_DQ = idesc_bf16_f32_ab(128, D, true, true);
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+  static_assert(COL_DK + D <= BW_TMEM_COLS, "tensor memory columns");
+};
+
+template <int D>
+__global__ void __launch_bounds__(BW_THREADS, 1)
+attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                   const BwdPlan pl) {
+  using C = BwCfg<D>;
+  // The 128-byte swizzle needs 1 KB-aligned tiles; the whole budget is used, so there is
+  // no slack to align by hand: the declaration asks for it and the kernel checks it.
+  extern __shared__ __align__(1024) uint8_t bw_smem[];
+  uint8_t* smem = bw_smem;
+  const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {
+    if (threadIdx.x == 0) record_error(DEVERR_BOUNDS);
+    return;
+  }
+  const uint32_t sK = sbase + C::K_OFF, sV = sbase + C::V_OFF, sDS = sbase + C::DS_OFF;
+  auto sQ = [&](int st) { return sbase + C::Q_OFF + (uint32_t)(2 * st) * C::TILE_BYTES; };
+  auto sDO = [&](int st) { return sbase + C::Q_OFF + (uint32_t)(2 * st + 1) * C::TILE_BYTES; };
+  const uint32_t bar0 = sbase + C::BAR_OFF;
+  const uint32_t bar_kv_full = bar0;
+  auto bar_q_full = [&](int st) { return bar0 + 8u * (1 + st); };
+  auto bar_q_empty = [&](int st) { return bar0 + 8u * (3 + st); };
+  const uint32_t bar_s_full = bar0 + 8u * 5, bar_dp_full = bar0 + 8u * 6, bar_p_ready = bar0 + 8u * 7,
+                 bar_ds_ready = bar0 + 8u * 8, bar_ds_free = bar0 + 8u * 9, bar_dq_full = bar0 + 8u * 10,
+                 bar_dq_free = bar0 + 8u * 11, bar_acc_done = bar0 + 8u * 12, bar_drain = bar0 + 8u * 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // Head-major: CTAs running together share one head's Q / dO stream through L2.
+  const int units_per_head = (int)(gridDim.x / pl.BH);
+  const int bh = blockIdx.x / units_per_head;
+  const KTile kt = decode_ktile(pl, blockIdx.x % units_per_head);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_kv_full, 1);
+    for (int st = 0; st < BW_NSTAGE; ++st) {
+      mbar_init(bar_q_full(st), 1 + 32);  // TMA transaction arrive + the producer's 32 lanes
+      mbar_init(bar_q_empty(st), 1);
+    }
+    mbar_init(bar_s_full, 1);
+    mbar_init(bar_dp_full, 1);
+    mbar_init(bar_p_ready, 256);
+    mbar_init(bar_ds_ready, 256);
+    mbar_init(bar_ds_free, 1);
+    mbar_init(bar_dq_full, 1);
+    mbar_init(bar_dq_free, 256);
+    mbar_init(bar_acc_done, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == BW_WARP_MMA) {
+    tmem_alloc(smem_u32(tmem_slot), BW_TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == BW_WARP_PRODUCER && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+    prefetch_tensormap(&tm_do);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  int T = 0;  // query tiles this CTA visits (the same walk in every role)
+  walk_q_tiles(pl, kt, [&](const Seg&, int64_t) { ++T; return true; });
+
+  if (warp >= 8) regs_decrease<BW_REGS_OTHER>();
+  if (warp == BW_WARP_PRODUCER) {
+    // ------------------------------------------------------------------ producer
+    if (T > 0) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar_kv_full, 2 * C::TILE_BYTES);
+        const int ky = (int)(kt.seg.row0 % kt.seg.stride);
+        const int kz = (int)(kt.seg.row0 / kt.seg.stride + kt.j0);
+        for (int b = 0; b < C::NBOX; ++b) {
+          tma_load_4d(sK + b * C::BOX_BYTES, &tm_k, bar_kv_full, 64 * b, ky, kz, bh);
+          tma_load_4d(sV + b * C::BOX_BYTES, &tm_v, bar_kv_full, 64 * b, ky, kz, bh);
+        }
+      }
+      int issued = 0;
+      walk_q_tiles(pl, kt, [&](const Seg& qs, int64_t i0) {
+        const int st = issued & 1;
+        const uint32_t ph = (uint32_t)(issued >> 1) & 1u;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_q_empty(st), ph ^ 1u, abort_flag))) return false;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar_q_full(st), 2 * C::TILE_BYTES);
+          const int qy = (int)(qs.row0 % qs.stride);
+          const int qz = (int)(qs.row0 / qs.stride + i0);
+          for (int b = 0; b < C::NBOX; ++b) {
+            tma_load_4d(sQ(st) + b * C::BOX_BYTES, &tm_q, bar_q_full(st), 64 * b, qy, qz, bh);
+            tma_load_4d(sDO(st) + b * C::BOX_BYTES, &tm_do, bar_q_full(st), 64 * b, qy, qz, bh);
+          }
+        }
+        float* l2s = reinterpret_cast<float*>(smem + C::LD_OFF + st * 2 * BWD_TILE * 4);
+        float* dls = l2s + BWD_TILE;
+        for (int r = lane; r < BWD_TILE; r += 32) {
+          const int64_t li = i0 + r;
+          float l2 = INFINITY, dd = 0.f;
+          if (li < qs.count) {
+            const int64_t idx = (int64_t)bh * pl.q_rows + qs.row0 + qs.stride * li;
+            const float l = pl.lse[idx];
+            if (l != -INFINITY) l2 = l * 1.4426950408889634f;
+            dd = pl.delta[idx];
+          }
+          l2s[r] = l2;
+          dls[r] = dd;
+        }
+        mbar_arrive(bar_q_full(st));
+        ++issued;
+        return true;
+      });
+      // Drain: every TMA load issued lands before the CTA's shared memory goes away.
+      if (lane == 0) {
+        mbar_wait_drain(bar_kv_full, 0);
+        for (int u = issued > BW_NSTAGE ? issued - BW_NSTAGE : 0; u < issued; ++u)
+          mbar_wait_drain(bar_q_full(u & 1), (uint32_t)(u >> 1) & 1u);
+      }
+      __syncwarp();
+    }
+  } else if (warp == BW_WARP_MMA) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (T > 0) {
+      const uint32_t hi = (1024u >> 4) | (1u << 14) | (2u << 29);  // SBO 1 KB, sm_100 version, 128B swizzle
+      auto lo_kmaj = [](uint32_t a) { return ((a & 0x3FFFFu) >> 4) | (1u << 16); };                     // LBO 16 B
+      auto lo_mnmaj = [](uint32_t a) { return ((a & 0x3FFFFu) >> 4) | ((uint32_t)(C::BOX_BYTES >> 4) << 16); };
+      auto desc = [&](uint32_t lo) { return ((uint64_t)hi << 32) | lo; };
+      // K-major k-step kk (16 elements): 32 B inside a 128 B row, the next box every 4 steps.
+      auto koff = [](int kk) { return (uint32_t)(((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4); };
+      // MN-major k-step: 16 rows of 128 B.
+      auto mnoff = [](int kk) { return (uint32_t)(kk * (2048 >> 4)); };
+      const uint32_t tS = tmem + C::COL_S, tDP = tmem + C::COL_DP, tDQ = tmem + C::COL_DQ,
+                     tDV = tmem + C::COL_DV, tDK = tmem + C::COL_DK;
+      const uint32_t lk = lo_kmaj(sK), lv = lo_kmaj(sV), lk_mn = lo_mnmaj(sK);
+      const uint32_t lds_k = lo_kmaj(sDS), lds_mn = lo_mnmaj(sDS);
+      auto wait_all = [&](uint32_t bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+      };
+      bool ok = wait_all(bar_kv_full, 0);
+      for (int i = 0; i < T && ok; ++i) {
+        const int st = i & 1;
+        const uint32_t ph = (uint32_t)(i >> 1) & 1u, pi = (uint32_t)i & 1u;
+        const uint32_t lq = lo_kmaj(sQ(st)), ldo = lo_kmaj(sDO(st));
+        const uint32_t lq_mn = lo_mnmaj(sQ(st)), ldo_mn = lo_mnmaj(sDO(st));
+        if (!(ok = wait_all(bar_q_full(st), ph))) break;
+        tc_fence_after_sync();
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ss(tS, desc(lk + koff(kk)), desc(lq + koff(kk)), C::IDESC_SS, kk > 0);
+          tc_commit(bar_s_full);
+        }
+        __syncwarp();
+        if (C::DQ_IN_DP && i > 0) {
+          if (!(ok = wait_all(bar_dq_free, pi ^ 1u))) break;
+          tc_fence_after_sync();
+        }
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ss(tDP, desc(lv + koff(kk)), desc(ldo + koff(kk)), C::IDESC_SS, kk > 0);
+          tc_commit(bar_dp_full);
+        }
+        __syncwarp();
+        if (!(ok = wait_all(bar_p_ready, pi))) break;
+        tc_fence_after_sync();
+        if (elect_one()) {
+          // P^T pairs: queries 0-63 in columns [0, 32), queries 64-127 in [64, 96).
+#pragma unroll
+          for (int kk = 0; kk < BWD_TILE / 16; ++kk)
+            mma_bf16_ts(tDV, tS + kk * 8 + (kk >= 4 ? 32 : 0), desc(ldo_mn + mnoff(kk)), C::IDESC_KMN,
+                        (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        __syncwarp();
+        if (!(ok = wait_all(bar_ds_ready, pi))) break;
+        tc_fence_after_sync();
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < BWD_TILE / 16; ++kk)
+            mma_bf16_ss(tDK, desc(lds_k + koff(kk)), desc(lq_mn + mnoff(kk)), C::IDESC_KMN,
+                        (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < BWD_TILE / 16; ++kk)
+            mma_bf16_ss(tDQ, desc(lds_mn + mnoff(kk)), desc(lk_mn + mnoff(kk)), C::IDESC_DQ, kk > 0);
+          tc_commit(bar_dq_full);
+          tc_commit(bar_ds_free);
+          tc_commit(bar_q_empty(st));
+          if (i == T - 1) tc_commit(bar_acc_done);
+        }
+        __syncwarp();
+      }
+      if (elect_one()) {
+        tc_commit(bar_drain);
+        mbar_wait_drain(bar_drain, 0);
+      }
+      __syncwarp();
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------------ math warpgroups
+    regs_increase<BW_REGS_MATH>();
+    const int g = warp >> 2;
+    const int row = threadIdx.x & 127;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const int c0 = 64 * g;  // this thread's query columns of S^T / dP^T
+    const uint32_t tS = tmem + C::COL_S + lane_off, tDP = tmem + C::COL_DP + lane_off,
+                   tDQ = tmem + C::COL_DQ + lane_off;
+    const int64_t jl = kt.j0 + row;
+    const bool kvalid = jl < kt.seg.count;
+    const int64_t tk = pl.k_tok0 + pl.k_tok_stride * (kt.seg.row0 + kt.seg.stride * jl);
+    const float sl2 = pl.scale_log2, scale = pl.scale;
+    uint8_t* ds_row = smem + C::DS_OFF + g * C::BOX_BYTES + row * 128;
+    int i = 0;
+    bool ok = true;
+    walk_q_tiles(pl, kt, [&](const Seg& qs, int64_t i0) {
+      const int st = i & 1;
+      const uint32_t ph = (uint32_t)(i >> 1) & 1u, pi = (uint32_t)i & 1u;
+      // Causal: query column c (token tq0 + tqs c) sees this key iff c >= lo.
+      const int64_t tqs = pl.q_tok_stride * qs.stride;
+      const int64_t tq0 = pl.q_tok0 + pl.q_tok_stride * (qs.row0 + qs.stride * i0);
+      int lo = 0;
+      if (!kvalid) lo = BWD_TILE;
+      else if (pl.causal && tk > tq0) {
+        const int64_t cmin = (tk - tq0 + tqs - 1) / tqs;
+        lo = cmin > BWD_TILE ? BWD_TILE : (int)cmin;
+      }
+      const bool nomask = __all_sync(0xffffffffu, lo <= c0);
+      const float* l2s = reinterpret_cast<const float*>(smem + C::LD_OFF + st * 2 * BWD_TILE * 4) + c0;
+      const float* dls = l2s + BWD_TILE;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar_q_full(st), ph, abort_flag)))) return false;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full, pi, abort_flag)))) return false;
+      tc_fence_after_sync();
+      uint32_t sr[64];
+      RA_TMEM_LD32(tS + c0, sr);
+      RA_TMEM_LD32(tS + c0 + 32, (sr + 32));
+      tmem_wait_ld();
+      RA_REG_FENCE32(sr);
+      RA_REG_FENCE32((sr + 32));
+      float p[64];
+#pragma unroll
+      for (int j = 0; j < 64; j += 4) {
+        const float4 L = *reinterpret_cast<const float4*>(l2s + j);
+        p[j + 0] = ex2_approx(fmaf(__uint_as_float(sr[j + 0]), sl2, -L.x));
+        p[j + 1] = ex2_approx(fmaf(__uint_as_float(sr[j + 1]), sl2, -L.y));
+        p[j + 2] = ex2_approx(fmaf(__uint_as_float(sr[j + 2]), sl2, -L.z));
+        p[j + 3] = ex2_approx(fmaf(__uint_as_float(sr[j + 3]), sl2, -L.w));
+      }
+      if (!nomask) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) p[j] = (c0 + j >= lo) ? p[j] : 0.f;
+      }
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(p[2 * j], p[2 * j + 1]);
+        RA_TMEM_ST32(tS + c0, pk);
+        tmem_wait_st();
+      }
+      tc_fence_before_sync();
+      mbar_arrive(bar_p_ready);
+
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_full, pi, abort_flag)))) return false;
+      tc_fence_after_sync();
+      RA_TMEM_LD32(tDP + c0, sr);
+      RA_TMEM_LD32(tDP + c0 + 32, (sr + 32));
+      tmem_wait_ld();
+      RA_REG_FENCE32(sr);
+      RA_REG_FENCE32((sr + 32));
+      if (i > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(bar_ds_free, pi ^ 1u, abort_flag)))) return false;
+      // dS^T row (this key) x 64 queries -> 8 chunks of 16 B, chunk ch at slot ch ^ (row % 8).
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        const float4 D0 = *reinterpret_cast<const float4*>(dls + 8 * ch);
+        const float4 D1 = *reinterpret_cast<const float4*>(dls + 8 * ch + 4);
+        const float dd[8] = {D0.x, D0.y, D0.z, D0.w, D1.x, D1.y, D1.z, D1.w};
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j0 = 8 * ch + 2 * e;
+          const float a = p[j0] * (__uint_as_float(sr[j0]) - dd[2 * e]) * scale;
+          const float b = p[j0 + 1] * (__uint_as_float(sr[j0 + 1]) - dd[2 * e + 1]) * scale;
+          w[e] = pack_bf16x2(a, b);
+        }
+        *reinterpret_cast<uint4*>(ds_row + ((ch ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar_ds_ready);
+
+      // dQ_i: thread = query row `row`, columns g d/2 .. g d/2 + d/2 - 1.
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar_dq_full, pi, abort_flag)))) return false;
+      tc_fence_after_sync();
+      const int64_t li = i0 + row;
+      const bool qvalid = li < qs.count;
+      float* dq_row = pl.dq + ((int64_t)bh * pl.q_rows + qs.row0 + qs.stride * li) * D + g * (D / 2);
+#pragma unroll
+      for (int cc = 0; cc < D / 64; ++cc) {
+        uint32_t r[32];
+        RA_TMEM_LD32(tDQ + g * (D / 2) + cc * 32, r);
+        tmem_wait_ld();
+        RA_REG_FENCE32(r);
+        if (qvalid) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            atomicAdd(reinterpret_cast<float4*>(dq_row + cc * 32 + 4 * j),
+                      make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                  __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
+        }
+      }
+      tc_fence_before_sync();
+      mbar_arrive(bar_dq_free);
+      ++i;
+      return true;
+    });
+
+    // ---- epilogue: dV and dK of this thread's key row, columns g d/2 .. g d/2 + d/2 - 1
+    if (ok && T > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_acc_done, 0, abort_flag));
+    if (ok) {
+      if (T > 0) tc_fence_after_sync();
+      const int64_t krow = kt.seg.row0 + kt.seg.stride * jl;
+      const int64_t off = ((int64_t)bh * pl.k_rows + krow) * D + g * (D / 2);
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const uint32_t tAcc = tmem + (m == 0 ? C::COL_DV : C::COL_DK) + lane_off + g * (D / 2);
+        void* dst = m == 0 ? pl.dv : pl.dk;
+#pragma unroll
+        for (int cc = 0; cc < D / 64; ++cc) {
+          uint32_t r[32];
+          if (T > 0) {
+            RA_TMEM_LD32(tAcc + cc * 32, r);
+            tmem_wait_ld();
+            RA_REG_FENCE32(r);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) r[j] = 0u;
+          }
+          if (!kvalid) continue;
+          if (pl.accumulate) {
+            float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(dst) + off + cc * 32);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              float4 a = o4[j];
+              a.x += __uint_as_float(r[4 * j]);
+              a.y += __uint_as_float(r[4 * j + 1]);
+              a.z += __uint_as_float(r[4 * j + 2]);
+              a.w += __uint_as_float(r[4 * j + 3]);
+              o4[j] = a;
+            }
+          } else {
+            uint4* o16 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + off + cc * 32);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              o16[j] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * j]), __uint_as_float(r[8 * j + 1])),
+                                  pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3])),
+                                  pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5])),
+                                  pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7])));
+          }
+        }
+      }
+    }
+  }
+
+  // ---- teardown: TMEM is released only after every tcgen05 operation has finished.
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == BW_WARP_MMA) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, BW_TMEM_COLS);
+  }
+}
+
+}  // namespace ra

@@ -243,6 +243,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
          | ((uint32_t)(M >> 4) << 24);          // M / 16
 }
 
+// As above with the A operand's major-ness too (bit 15: A MN-major, read from shared memory).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_ab(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return idesc_bf16_f32(M, N, b_mn_major) | ((a_mn_major ? 1u : 0u) << 15);
+}
+
+// Orders this thread's generic-proxy shared-memory writes before later async-proxy reads
+// (tensor-core operand fetches) of the same bytes.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand. Start address, leading
 // and stride byte offsets are stored divided by 16; bit 46 is the sm_100 descriptor
 // version; bits 61-63 = 2 select the 128B swizzle.

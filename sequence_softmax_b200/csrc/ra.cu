@@ -8,8 +8,10 @@
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
 #include "merge.cuh"
+#include "bwd.cuh"
+#include "bwd_tc.cuh"
 
-#define RA_ABI_VERSION 1
+#define RA_ABI_VERSION 2
 
 namespace ra {
 
@@ -107,6 +109,69 @@ ra_status launch_attention(const Plan& pl, ra_dtype dt, int S, cudaStream_t stre
   if (gx > 0x7FFFFFFFll || pl.P > 65535 || pl.BH > 65535) return RA_ERR_UNSUPPORTED;
   dim3 grid((unsigned)gx, (unsigned)pl.P, (unsigned)pl.BH);
   attn_fwd_simt_f32_kernel<<<grid, SIMT_WARPS * 32, 0, stream>>>(pl, rows_per_pos);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+// Sets the dynamic shared-memory opt-in of `fn` once per device.
+template <class K>
+ra_status set_smem_attr_once(K* fn, int bytes, bool (&done)[64]) {
+  static std::mutex mu;
+  std::lock_guard<std::mutex> g(mu);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RA_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return RA_ERR_UNSUPPORTED;
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+      return RA_ERR_CUDA;
+    done[dev] = true;
+  }
+  return RA_OK;
+}
+
+template <int D>
+ra_status launch_bwd_tc(const BwdPlan& pl, int S, cudaStream_t stream) {
+  using C = BwCfg<D>;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_tile_map(&mq, pl.q, pl.BH, pl.q_rows, D, S) || !make_tile_map(&mk, pl.k, pl.BH, pl.k_rows, D, S) ||
+      !make_tile_map(&mv, pl.v, pl.BH, pl.k_rows, D, S) || !make_tile_map(&mdo, pl.d_o, pl.BH, pl.q_rows, D, S))
+    return RA_ERR_CUDA;
+  static bool done[64] = {};
+  ra_status st = set_smem_attr_once(attn_bwd_tc_kernel<D>, C::SMEM_BYTES, done);
+  if (st != RA_OK) return st;
+  const int64_t nkt = (pl.k_seg_len + BWD_TILE - 1) / BWD_TILE;
+  const int64_t grid = nkt * (int64_t)pl.P * num_segments(pl.layout) * pl.BH;
+  if (grid <= 0) return RA_OK;
+  if (grid > 0x7FFFFFFFll) return RA_ERR_UNSUPPORTED;
+  attn_bwd_tc_kernel<D><<<(unsigned)grid, BW_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, pl);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+// The gradient kernels of one plan: the tensor-core kernel for bf16, the two fp32 kernels
+// otherwise. S = row spacing of the striped view (P) or 1.
+ra_status launch_backward(const BwdPlan& pl, ra_dtype dt, int S, cudaStream_t stream) {
+  if (dt == RA_BF16) {
+    if (pl.d == 128) return launch_bwd_tc<128>(pl, S, stream);
+    if (pl.d == 64) return launch_bwd_tc<64>(pl, S, stream);
+    return RA_ERR_UNSUPPORTED;
+  }
+  const int64_t krows = pl.k_seg_len * num_segments(pl.layout);
+  const int64_t qrows = pl.q_seg_len * num_segments(pl.layout);
+  const int64_t gk = (krows + SIMT_WARPS - 1) / SIMT_WARPS, gq = (qrows + SIMT_WARPS - 1) / SIMT_WARPS;
+  if (gk > 0x7FFFFFFFll || gq > 0x7FFFFFFFll || pl.P > 65535 || pl.BH > 65535) return RA_ERR_UNSUPPORTED;
+  if (gk > 0) bwd_dkdv_simt_f32_kernel<<<dim3((unsigned)gk, pl.P, pl.BH), SIMT_WARPS * 32, 0, stream>>>(pl, krows);
+  if (gq > 0) bwd_dq_simt_f32_kernel<<<dim3((unsigned)gq, pl.P, pl.BH), SIMT_WARPS * 32, 0, stream>>>(pl, qrows);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+ra_status launch_delta(const void* o, const void* d_o, ra_dtype dt, int64_t rows, int d, float* delta,
+                       float* zero_rows, cudaStream_t stream) {
+  if (rows == 0) return RA_OK;
+  int64_t blocks = (rows + DELTA_THREADS / 8 - 1) / (DELTA_THREADS / 8);
+  if (blocks > (1ll << 20)) blocks = 1ll << 20;
+  if (dt == RA_BF16)
+    bwd_delta_kernel<true><<<(unsigned)blocks, DELTA_THREADS, 0, stream>>>(o, d_o, rows, d, delta, zero_rows);
+  else
+    bwd_delta_kernel<false><<<(unsigned)blocks, DELTA_THREADS, 0, stream>>>(o, d_o, rows, d, delta, zero_rows);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
@@ -241,6 +306,97 @@ ra_status ra_ring_forward(const void* q, const void* k, const void* v, ra_dtype 
   pl.scale_log2 = scale * 1.4426950408889634f;
   const int S = layout == RA_LAYOUT_STRIPED ? n_chunks : 1;
   return launch_attention(pl, dt, S, stream);
+}
+
+ra_status ra_backward_delta(const void* o, const void* d_o, ra_dtype dt, int64_t rows, int d, float* delta,
+                            cudaStream_t stream) {
+  if (rows < 0) return RA_ERR_INVALID_ARG;
+  ra_status st = check_dtype_d(dt, d);
+  if (st != RA_OK) return st;
+  if (rows == 0) return RA_OK;
+  if (!o || !d_o || !delta || !aligned16(o) || !aligned16(d_o) || (reinterpret_cast<uintptr_t>(delta) & 3u))
+    return RA_ERR_INVALID_ARG;
+  return launch_delta(o, d_o, dt, rows, d, delta, nullptr, stream);
+}
+
+ra_status ra_partial_backward(const void* q, const void* k, const void* v, const void* d_o, const float* lse,
+                              const float* delta, ra_dtype dt, int B, int H, int64_t Lq, int64_t Lk, int d,
+                              float scale, int causal, int64_t q_tok0, int64_t q_tok_stride, int64_t k_tok0,
+                              int64_t k_tok_stride, float* dq_acc, float* dk_acc, float* dv_acc,
+                              cudaStream_t stream) {
+  if (B < 0 || H < 0 || Lq < 0 || Lk < 0) return RA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return RA_ERR_INVALID_ARG;
+  if (q_tok_stride < 1 || k_tok_stride < 1) return RA_ERR_INVALID_ARG;
+  ra_status st = check_dtype_d(dt, d);
+  if (st != RA_OK) return st;
+  if ((int64_t)B * H > 0x7FFFFFFF) return RA_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || Lq == 0 || Lk == 0) return RA_OK;
+  if (!q || !k || !v || !d_o || !lse || !delta || !dq_acc || !dk_acc || !dv_acc) return RA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(d_o) || !aligned16(dq_acc) ||
+      !aligned16(dk_acc) || !aligned16(dv_acc) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(delta) & 3u))
+    return RA_ERR_INVALID_ARG;
+  BwdPlan pl{};
+  pl.q = q; pl.k = k; pl.v = v; pl.d_o = d_o; pl.lse = lse; pl.delta = delta;
+  pl.dq = dq_acc; pl.dk = dk_acc; pl.dv = dv_acc;
+  pl.BH = B * H; pl.d = d; pl.P = 1; pl.layout = RA_LAYOUT_CONTIGUOUS; pl.causal = causal;
+  pl.accumulate = 1; pl.dkdv_bf16 = 0;
+  pl.q_rows = Lq; pl.k_rows = Lk; pl.q_seg_len = Lq; pl.k_seg_len = Lk;
+  pl.q_tok0 = q_tok0; pl.q_tok_stride = q_tok_stride; pl.k_tok0 = k_tok0; pl.k_tok_stride = k_tok_stride;
+  pl.scale = scale;
+  pl.scale_log2 = scale * 1.4426950408889634f;
+  return launch_backward(pl, dt, 1, stream);
+}
+
+int64_t ra_ring_backward_workspace_bytes(ra_dtype dt, int B, int H, int64_t N, int d) {
+  if (B < 0 || H < 0 || N < 0 || d < 1) return -1;
+  const int64_t rows = (int64_t)B * H * N;
+  return dt == RA_BF16 ? rows * (d + 1) * 4 : rows * 4;
+}
+
+ra_status ra_ring_backward(const void* q, const void* k, const void* v, const void* o, const void* d_o,
+                           const float* lse, ra_dtype dt, int B, int H, int64_t N, int d, float scale,
+                           int n_chunks, int causal, ra_layout layout, void* dq, void* dk, void* dv,
+                           void* workspace, int64_t workspace_bytes, cudaStream_t stream) {
+  if (B < 0 || H < 0 || N < 0 || n_chunks < 1) return RA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return RA_ERR_INVALID_ARG;
+  if (layout != RA_LAYOUT_CONTIGUOUS && layout != RA_LAYOUT_STRIPED && layout != RA_LAYOUT_ZIGZAG)
+    return RA_ERR_INVALID_ARG;
+  const int64_t parts = layout == RA_LAYOUT_ZIGZAG ? 2 * (int64_t)n_chunks : n_chunks;
+  if (N % parts != 0) return RA_ERR_INVALID_ARG;
+  ra_status st = check_dtype_d(dt, d);
+  if (st != RA_OK) return st;
+  if ((int64_t)B * H > 0x7FFFFFFF) return RA_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || N == 0) return RA_OK;
+  if (workspace_bytes < ra_ring_backward_workspace_bytes(dt, B, H, N, d)) return RA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !d_o || !lse || !dq || !dk || !dv || !workspace) return RA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(d_o) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return RA_ERR_INVALID_ARG;
+  const int64_t rows = (int64_t)B * H * N;
+  const bool bf = dt == RA_BF16;
+  float* dq_acc = bf ? static_cast<float*>(workspace) : static_cast<float*>(dq);
+  float* delta = bf ? static_cast<float*>(workspace) + rows * d : static_cast<float*>(workspace);
+  st = launch_delta(o, d_o, dt, rows, d, delta, bf ? dq_acc : nullptr, stream);
+  if (st != RA_OK) return st;
+  BwdPlan pl{};
+  pl.q = q; pl.k = k; pl.v = v; pl.d_o = d_o; pl.lse = lse; pl.delta = delta;
+  pl.dq = dq_acc; pl.dk = dk; pl.dv = dv;
+  pl.BH = B * H; pl.d = d; pl.P = n_chunks; pl.layout = layout; pl.causal = causal;
+  pl.accumulate = 0; pl.dkdv_bf16 = bf ? 1 : 0;
+  pl.q_rows = N; pl.k_rows = N;
+  pl.q_seg_len = pl.k_seg_len = N / parts;
+  pl.q_tok0 = 0; pl.q_tok_stride = 1; pl.k_tok0 = 0; pl.k_tok_stride = 1;
+  pl.scale = scale;
+  pl.scale_log2 = scale * 1.4426950408889634f;
+  st = launch_backward(pl, dt, layout == RA_LAYOUT_STRIPED ? n_chunks : 1, stream);
+  if (st != RA_OK || !bf) return st;
+  int64_t blocks = (rows * d / 4 + 255) / 256;
+  if (blocks > (1ll << 20)) blocks = 1ll << 20;
+  f32_to_bf16_kernel<<<(unsigned)blocks, 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), rows * d / 4);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -7,6 +7,9 @@
   dV_j = sum of dO over the queries that see key j, divided by each query's count.
 * ``pin_ring_equals_definition``: the ring backward equals the definition for every layout,
   causal and not, and for random visiting orders.
+* ``pin_partials_sum_to_definition``: partial_backward over every (query position, KV chunk)
+  pair of a contiguous and a striped split, with the final lse and D, sums to the definition.
+* ``pin_rows_equal_definition``: backward_rows equals the definition at the chosen rows.
 """
 
 from __future__ import annotations
@@ -125,4 +128,53 @@ def pin_ring_equals_definition(Bk):
     return _all(checks)
 
 
-ALL_BACKWARD_PINS = [pin_autograd, pin_finite_differences, pin_closed_forms, pin_ring_equals_definition]
+def pin_partials_sum_to_definition(Bk):
+    import oracle as Fw
+    checks = []
+    r = np.random.default_rng(15)
+    B, H, N, d, P = 2, 1, 40, 8, 4
+    q, k, v, do = (r.standard_normal((B, H, N, d)) for _ in range(4))
+    for causal in (False, True):
+        want = Bk.attention_backward(q, k, v, do, d ** -0.5, causal)
+        o, lse = Fw.attention(q, k, v, d ** -0.5, causal)
+        dd = Bk.delta(o, do)
+        for layout in ("contiguous", "striped"):
+            got = [np.zeros_like(x) for x in want]
+            for pq in range(P):
+                for pk in range(P):
+                    if layout == "contiguous":
+                        iq, ik = np.arange(pq * N // P, (pq + 1) * N // P), np.arange(pk * N // P, (pk + 1) * N // P)
+                        args = (int(iq[0]), 1, int(ik[0]), 1)
+                    else:
+                        iq, ik = np.arange(pq, N, P), np.arange(pk, N, P)
+                        args = (pq, P, pk, P)
+                    g = Bk.partial_backward(q[:, :, iq], k[:, :, ik], v[:, :, ik], do[:, :, iq], lse[:, :, iq],
+                                            dd[:, :, iq], d ** -0.5, causal, *args)
+                    got[0][:, :, iq] += g[0]
+                    got[1][:, :, ik] += g[1]
+                    got[2][:, :, ik] += g[2]
+            checks += [_close(a, b) for a, b in zip(got, want)]
+    return _all(checks)
+
+
+def pin_rows_equal_definition(Bk):
+    checks = []
+    r = np.random.default_rng(16)
+    B, H, N, d = 1, 3, 50, 8
+    q, k, v, do = (r.standard_normal((B, H, N, d)) for _ in range(4))
+    rows_q, rows_k = np.array([0, 7, 49]), np.array([0, 1, 30, 49])
+    for causal in (False, True):
+        dq, dk, dv = Bk.attention_backward(q, k, v, do, d ** -0.5, causal)
+        heads = [(0, 2), (0, 0)]
+        gq, gk, gv = Bk.backward_rows(q, k, v, do, d ** -0.5, causal, rows_q, rows_k, heads=heads)
+        for n, (b, h) in enumerate(heads):
+            checks += [_close(gq[n], dq[b, h, rows_q]), _close(gk[n], dk[b, h, rows_k]), _close(gv[n], dv[b, h, rows_k])]
+        gq, gk, _ = Bk.backward_rows(q, k, v, do, d ** -0.5, causal, rows_q, [], heads=heads)
+        checks.append((gk.size == 0, "no key rows asked"))
+        for n, (b, h) in enumerate(heads):
+            checks.append(_close(gq[n], dq[b, h, rows_q]))
+    return _all(checks)
+
+
+ALL_BACKWARD_PINS = [pin_autograd, pin_finite_differences, pin_closed_forms, pin_ring_equals_definition,
+                     pin_partials_sum_to_definition, pin_rows_equal_definition]

@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.ra_abi_version() == 1
+    assert lib.ra_abi_version() == 2
     for code in range(6):
         s = binding.status_string(code)
         assert s.startswith("RA_")
@@ -124,6 +124,73 @@ def test_merge_rejects(lib, kw, code):
 
 def test_merge_empty_is_noop(lib):
     assert _merge(lib, rows=0) == binding.RA_OK
+
+
+def _ring_bwd(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, d_o=FAKE, lse=FAKE, dt=1, B=1, H=2, N=256, d=128, scale=0.1,
+             n_chunks=2, causal=1, layout=2, dq=FAKE, dk=FAKE, dv=FAKE, ws=FAKE, ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return lib.ra_ring_backward(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_chunks=0), binding.RA_ERR_INVALID_ARG),
+    (dict(N=256, n_chunks=3), binding.RA_ERR_INVALID_ARG),           # zig-zag needs N % 2P == 0
+    (dict(layout=9), binding.RA_ERR_INVALID_ARG),
+    (dict(scale=0.0), binding.RA_ERR_INVALID_ARG),
+    (dict(d=96), binding.RA_ERR_UNSUPPORTED),
+    (dict(ws_bytes=1000), binding.RA_ERR_INVALID_ARG),               # workspace too small
+    (dict(ws=None), binding.RA_ERR_INVALID_ARG),
+    (dict(lse=ctypes.c_void_p(0x10002)), binding.RA_ERR_INVALID_ARG),
+    (dict(dk=ctypes.c_void_p(0x10004)), binding.RA_ERR_INVALID_ARG),
+])
+def test_ring_backward_rejects(lib, kw, code):
+    assert _ring_bwd(lib, **kw) == code
+
+
+def test_ring_backward_workspace_size(lib):
+    f = lib.ra_ring_backward_workspace_bytes
+    assert f(1, 1, 2, 256, 128) == 2 * 256 * 129 * 4      # fp32 dQ accumulator + D
+    assert f(0, 1, 2, 256, 16) == 2 * 256 * 4             # D only
+    assert f(1, -1, 2, 256, 128) == -1
+    assert _ring_bwd(lib, ws_bytes=f(1, 1, 2, 256, 128) - 1) == binding.RA_ERR_INVALID_ARG
+    assert _ring_bwd(lib, N=0) == binding.RA_OK
+
+
+def _partial_bwd(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, d_o=FAKE, lse=FAKE, delta=FAKE, dt=1, B=1, H=1, Lq=128, Lk=128, d=64,
+             scale=0.1, causal=1, q_tok0=0, q_ts=1, k_tok0=0, k_ts=1, dq=FAKE, dk=FAKE, dv=FAKE, stream=None)
+    a.update(kw)
+    return lib.ra_partial_backward(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Lk=-1), binding.RA_ERR_INVALID_ARG),
+    (dict(q_ts=0), binding.RA_ERR_INVALID_ARG),
+    (dict(d=32), binding.RA_ERR_UNSUPPORTED),
+    (dict(delta=None), binding.RA_ERR_INVALID_ARG),
+    (dict(dq=ctypes.c_void_p(0x10008)), binding.RA_ERR_INVALID_ARG),
+    (dict(causal=3), binding.RA_ERR_INVALID_ARG),
+])
+def test_partial_backward_rejects(lib, kw, code):
+    assert _partial_bwd(lib, **kw) == code
+
+
+def test_partial_backward_empty_is_noop(lib):
+    assert _partial_bwd(lib, Lq=0) == binding.RA_OK
+    assert _partial_bwd(lib, Lk=0) == binding.RA_OK
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(rows=-1), binding.RA_ERR_INVALID_ARG),
+    (dict(d=96), binding.RA_ERR_UNSUPPORTED),
+    (dict(delta=None), binding.RA_ERR_INVALID_ARG),
+    (dict(rows=0), binding.RA_OK),
+])
+def test_backward_delta_rejects(lib, kw, code):
+    a = dict(o=FAKE, d_o=FAKE, dt=1, rows=16, d=128, delta=FAKE, stream=None)
+    a.update(kw)
+    assert lib.ra_backward_delta(*a.values()) == code
 
 
 def test_product_path_does_not_reach_the_oracle():

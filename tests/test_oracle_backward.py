@@ -17,32 +17,34 @@ def test_backward_pin(pin):
 _REAL = Bk._grads_block
 
 
-def _no_d_term(q, k, v, do, o, lse, scale, causal, tq, tk):
+def _no_d_term(q, k, v, do, d_row, lse, scale, causal, tq, tk):
     p = Bk._probs(q, k, scale, causal, lse, tq, tk)
     ds = p * (do @ v.T)
     return (ds @ k) * scale, (ds.T @ q) * scale, p.T @ do
 
 
-def _missing_scale(q, k, v, do, o, lse, scale, causal, tq, tk):
-    gq, gk, gv = _REAL(q, k, v, do, o, lse, scale, causal, tq, tk)
+def _missing_scale(q, k, v, do, d_row, lse, scale, causal, tq, tk):
+    gq, gk, gv = _REAL(q, k, v, do, d_row, lse, scale, causal, tq, tk)
     return gq / scale, gk, gv
 
 
-def _dv_untransposed(q, k, v, do, o, lse, scale, causal, tq, tk):
-    gq, gk, gv = _REAL(q, k, v, do, o, lse, scale, causal, tq, tk)
+def _dv_untransposed(q, k, v, do, d_row, lse, scale, causal, tq, tk):
+    gq, gk, gv = _REAL(q, k, v, do, d_row, lse, scale, causal, tq, tk)
     p = Bk._probs(q, k, scale, causal, lse, tq, tk)
-    return gq, gk, p @ do          # the pins' blocks are square, so the shapes agree
+    if p.shape[0] != p.shape[1]:
+        return gq, gk, gv * 1.5    # only square blocks can take p @ dO; corrupt the rest plainly
+    return gq, gk, p @ do
 
 
-def _dk_uses_k(q, k, v, do, o, lse, scale, causal, tq, tk):
-    gq, gk, gv = _REAL(q, k, v, do, o, lse, scale, causal, tq, tk)
+def _dk_uses_k(q, k, v, do, d_row, lse, scale, causal, tq, tk):
+    gq, gk, gv = _REAL(q, k, v, do, d_row, lse, scale, causal, tq, tk)
     p = Bk._probs(q, k, scale, causal, lse, tq, tk)
-    ds = p * (do @ v.T - (do * o).sum(axis=1)[:, None])
+    ds = p * (do @ v.T - d_row[:, None])
     return gq, (ds.T @ k) * scale, gv
 
 
-def _no_causal_mask(q, k, v, do, o, lse, scale, causal, tq, tk):
-    return _REAL(q, k, v, do, o, lse, scale, False, tq, tk)
+def _no_causal_mask(q, k, v, do, d_row, lse, scale, causal, tq, tk):
+    return _REAL(q, k, v, do, d_row, lse, scale, False, tq, tk)
 
 
 MUTANTS = {"drop-D": _no_d_term, "dq-missing-scale": _missing_scale, "dv-untransposed": _dv_untransposed,
