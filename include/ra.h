@@ -185,6 +185,35 @@ ra_status ra_ring_backward(const void* q, const void* k, const void* v, const vo
                            int n_chunks, int causal, ra_layout layout, void* dq, void* dk, void* dv,
                            void* workspace, int64_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * ra_ring_backward_noalloc -- ra_ring_backward for callers that must not allocate device
+ * memory themselves. Examples: a plugin or custom operator inside another runtime that hands
+ * it device pointers but owns every byte of the GPU through its own pool allocator (a raw
+ * cudaMalloc there takes memory the pool counts as free), or a latency-critical loop where
+ * cudaMalloc/cudaFree, which may synchronise the whole device, cannot run. The paper has no
+ * counterpart: this is an interface convenience, not part of the method.
+ *
+ * The scratch (the fp32 dQ accumulator and D) lives in one static device array of
+ * RA_NOALLOC_SCRATCH_BYTES bytes inside the library. Every GPU that loads the library holds
+ * it until the process exits. Problems whose ra_ring_backward_workspace_bytes() exceeds it
+ * return RA_ERR_UNSUPPORTED without launching anything (at d = 128 in bf16 the limit is
+ * B*H*N <= 130055 rows; fp32 needs only 4 bytes per row).
+ *
+ * The first call on a device looks up the array's device address, with that device current,
+ * and keeps it; make that first call before any stream capture. All calls on a device share
+ * the one array: two calls whose work overlaps on the GPU (different streams, or different
+ * host threads without ordering) race on it and corrupt each other's gradients, so order
+ * them on one stream or synchronise between them. Nothing needs clearing by the caller: each
+ * call zeroes the part of the array that must start at zero. Arguments, layouts and outputs
+ * are those of ra_ring_backward.
+ */
+#define RA_NOALLOC_SCRATCH_BYTES (64ll * 1024 * 1024)
+ra_status ra_ring_backward_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                   const void* d_o, const float* lse, ra_dtype dt, int B, int H,
+                                   int64_t N, int d, float scale, int n_chunks, int causal,
+                                   ra_layout layout, void* dq, void* dk, void* dv,
+                                   cudaStream_t stream);
+
 /* Static, human-readable name of a status code (never NULL). */
 const char* ra_status_string(ra_status status);
 

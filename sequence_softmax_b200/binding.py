@@ -35,6 +35,8 @@ SIGNATURES = {
     "ra_ring_backward_workspace_bytes": (_i64, [_i32, _i32, _i32, _i64, _i32]),
     "ra_ring_backward": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i64, _i32, _f32, _i32, _i32,
                                 _i32, _vp, _vp, _vp, _vp, _i64, _vp]),
+    "ra_ring_backward_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i64, _i32, _f32, _i32,
+                                        _i32, _i32, _vp, _vp, _vp, _vp]),
     "ra_status_string": (ctypes.c_char_p, [_i32]),
     "ra_get_device_error": (_i32, [_vp]),
     "ra_selftest_wait_timeout": (_i32, [_i64, _vp]),
@@ -282,4 +284,34 @@ def ring_backward(q, k, v, o, d_o, lse, n_chunks: int, causal: bool = False, lay
                                  workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                  _stream_ptr(stream))
     _check(st, "ra_ring_backward")
+    return dq, dk, dv
+
+
+def ring_backward_noalloc(q, k, v, o, d_o, lse, n_chunks: int, causal: bool = False, layout: str = "contiguous",
+                          scale: float | None = None, out=None, stream=None):
+    """``ring_backward`` through the entry point that allocates nothing on the device.
+
+    For callers that cannot allocate device memory: the library's static scratch array
+    replaces the workspace. Pass ``out`` = (dq, dk, dv) preallocated tensors to allocate
+    nothing here either. Calls on one device must not overlap on the GPU (they share the
+    scratch); problems larger than the array raise RaError(RA_ERR_UNSUPPORTED).
+    """
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (d_o, "d_o"), (lse, "lse")):
+        _dev(t, n)
+    B, H, N, d = q.shape
+    if any(t.shape != q.shape or t.dtype != q.dtype for t in (k, v, o, d_o)):
+        raise ValueError("q, k, v, o, d_o must share shape [B, H, N, d] and dtype")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N):
+        raise ValueError("lse must be float32 [B, H, N]")
+    if layout not in LAYOUTS:
+        raise ValueError(f"layout must be one of {sorted(LAYOUTS)}")
+    scale = d ** -0.5 if scale is None else float(scale)
+    dq, dk, dv = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)) if out is None else out
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _dev(t, n)
+    st = load().ra_ring_backward_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), d_o.data_ptr(),
+                                         lse.data_ptr(), _dtype_code(q), B, H, N, d, scale, int(n_chunks),
+                                         int(bool(causal)), LAYOUTS[layout], dq.data_ptr(), dk.data_ptr(),
+                                         dv.data_ptr(), _stream_ptr(stream))
+    _check(st, "ra_ring_backward_noalloc")
     return dq, dk, dv

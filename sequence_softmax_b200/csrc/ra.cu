@@ -400,3 +400,46 @@ ra_status ra_ring_backward(const void* q, const void* k, const void* v, const vo
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------
+// ra_ring_backward_noalloc: the workspace of ra_ring_backward in a static device array, so
+// that callers who cannot allocate device memory still get the backward pass.
+// ------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[RA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of this device's copy of g_noalloc_scratch (host code only sees a
+// host-side stand-in for the name). Looked up once per device, with that device current.
+ra_status noalloc_scratch(void** out) {
+  static void* addr[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RA_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return RA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> g(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return RA_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return RA_OK;
+}
+
+}  // namespace
+
+extern "C" ra_status ra_ring_backward_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                              const void* d_o, const float* lse, ra_dtype dt, int B, int H,
+                                              int64_t N, int d, float scale, int n_chunks, int causal,
+                                              ra_layout layout, void* dq, void* dk, void* dv,
+                                              cudaStream_t stream) {
+  const int64_t need = ra_ring_backward_workspace_bytes(dt, B, H, N, d);
+  if (need < 0) return RA_ERR_INVALID_ARG;
+  if (need > RA_NOALLOC_SCRATCH_BYTES) return RA_ERR_UNSUPPORTED;
+  void* ws = nullptr;
+  const ra_status st = noalloc_scratch(&ws);
+  if (st != RA_OK) return st;
+  return ra_ring_backward(q, k, v, o, d_o, lse, dt, B, H, N, d, scale, n_chunks, causal, layout, dq, dk, dv, ws,
+                          RA_NOALLOC_SCRATCH_BYTES, stream);
+}
