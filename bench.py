@@ -1,4 +1,5 @@
-"""Benchmark: ring-attention forward TFLOP/s on B200 (bf16), % of tensor peak; merge HBM GB/s.
+"""Benchmark: ring-attention forward TFLOP/s on B200 (bf16), % of tensor peak; merge HBM GB/s;
+backward TFLOP/s.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
@@ -11,6 +12,9 @@ N(0, 1)), resident in HBM and 6.4 GB in total, so they exceed the 126 MB L2 betw
 Rank 0 prints one JSON line. With N > 1 (torchrun) every rank runs an independent replica
 of the workload with its own seed (weak scaling, no collective on the data path); time is
 the max over ranks of CUDA-event time.
+
+Sub-measurements in the same line: "merge" (ra_merge, HBM-bound) and "backward"
+(ra_ring_backward on the 128K-token zig-zag workload).
 
 --impl reference times the fp64 CPU oracle on this host's cores on a bounded sample of the
 same workload (rows of one head against all their visible keys) in the same unit.
@@ -36,7 +40,10 @@ PROFILE_JSON = os.path.join(ROOT, "profiles", "counters.json")
 KERNEL_SOURCES = {
     "attn_fwd_tc": ["sequence_softmax_b200/csrc/attn_tc.cuh", "sequence_softmax_b200/csrc/common.cuh"],
     "merge": ["sequence_softmax_b200/csrc/merge.cuh"],
+    "attn_bwd_tc": ["sequence_softmax_b200/csrc/bwd_tc.cuh", "sequence_softmax_b200/csrc/bwd.cuh",
+                    "sequence_softmax_b200/csrc/common.cuh"],
 }
+BWD_WORKLOAD = "seq128k-d128-causal-zigzag16"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "source": "fallback"}
 
@@ -54,6 +61,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     ap.add_argument("--merge-rows", type=int, default=8 * (1 << 20),
                     help="rows of the merge workload (smaller values for profiler captures)")
+    ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--bwd-workload", default=BWD_WORKLOAD)
+    ap.add_argument("--bwd-steps", type=int, default=3)
     return ap.parse_args()
 
 
@@ -319,6 +329,10 @@ def main():
     del q, k, v
     torch.cuda.empty_cache()
 
+    if not a.no_backward:
+        line["backward"] = bench_backward(binding, torch, dev, pk, a, rank)
+        torch.cuda.empty_cache()
+
     if rank == 0 and not a.no_cpu_baseline and world == 1:
         tf, el, nr, threads = oracle_sample(w, a.cpu_seconds)
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
@@ -358,6 +372,53 @@ def bench_merge(binding, torch, dev, pk, a):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "traffic": traffic,
                          "peak_source": f"{pk['source']} copy"}}
+
+
+def bench_backward(binding, torch, dev, pk, a, rank):
+    """ra_ring_backward on its own workload: dQ, dK, dV of the forward's output for a seeded
+    upstream gradient. FLOPs = 2.5x the forward's (five GEMMs per visible pair instead of two)."""
+    from sequence_softmax_b200.inputs import WORKLOADS, make_qkv, workload_qkv
+    w = WORKLOADS[a.bwd_workload]
+    q, k, v = workload_qkv(w, device=dev, batch_offset=rank)
+    do = make_qkv(w.B, w.H, w.N, w.d, w.torch_dtype, seed=1000 + rank, device=dev)[0]
+    o, lse = binding.ring_forward(q, k, v, w.n_chunks, w.causal, w.layout)
+    ws = torch.empty(binding.ring_backward_workspace_bytes(q.dtype, w.B, w.H, w.N, w.d), device=dev,
+                     dtype=torch.uint8)
+    grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+
+    def step():
+        binding.ring_backward(q, k, v, o, do, lse, w.n_chunks, w.causal, w.layout, workspace=ws, out=grads)
+
+    step()
+    torch.cuda.synchronize()
+    if binding.get_device_error() != binding.RA_OK:
+        raise RuntimeError("device error in the backward warm-up")
+    stream = torch.cuda.current_stream()
+    # one ra_ring_backward call per timed step, on the stream its kernels are launched on
+    kernel_ms = []
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    for _ in range(a.bwd_steps):
+        s.record(stream)
+        step()
+        e.record(stream)
+        e.synchronize()
+        kernel_ms.append(s.elapsed_time(e))
+    if binding.get_device_error() != binding.RA_OK:
+        raise RuntimeError("device error in the timed backward")
+    ms = statistics.median(kernel_ms)
+    flops = 2.5 * w.flops()
+    tf = flops / (ms / 1e3) / 1e12
+    peak = pk["bf16_tflops"]
+    traffic = stored_traffic("attn_bwd_tc", w.name, w.B * w.H * w.N)
+    return {"value": tf, "unit": "TFLOP/s", "ms_per_step": ms, "steps": a.bwd_steps,
+            "workload": workload_config(w), "flops_per_step": flops,
+            "gpu_launches_per_step": 3,
+            "note": "one step = ra_ring_backward: D + zeroed dQ accumulator, the gradient kernel, dQ to bf16",
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                         "traffic": traffic, "peak_source": f"{pk['source']} bf16 burst",
+                         "kernel": "attn_bwd_tc_kernel<128> (+ 2 bandwidth-bound launches, ~1% of the step)"},
+            "wall_s": time.time() - t0}
 
 
 def bench_e2e(binding, torch, w, q, k, v, world, a):

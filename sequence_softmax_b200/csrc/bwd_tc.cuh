@@ -13,8 +13,9 @@
 //   dP^T = V dO_i^T            (same form)
 //   P^T  = exp2(S^T scale log2e - lse_i log2e), masked; bf16 into the S columns of TMEM
 //   dV  += P^T dO_i            (A = P^T from TMEM, B = dO_i MN-major)
-//   dS^T = P^T (dP^T - D_i) scale, bf16 into a 128B-swizzled shared-memory tile
-//   dK  += dS^T Q_i            (A = dS^T K-major, B = Q_i MN-major)
+//   dS^T = P^T (dP^T - D_i) scale, bf16 into the dP columns of TMEM and into a
+//                              128B-swizzled shared-memory tile
+//   dK  += dS^T Q_i            (A = dS^T from TMEM, B = Q_i MN-major)
 //   dQ_i = dS K                (A = the same dS tile read MN-major, B = K MN-major)
 // so each (query tile, key tile) pair costs five 128 x 128 x d GEMMs and one exponential per
 // score, and P and dS never leave the SM.
@@ -225,7 +226,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const uint32_t tS = tmem + C::COL_S, tDP = tmem + C::COL_DP, tDQ = tmem + C::COL_DQ,
                      tDV = tmem + C::COL_DV, tDK = tmem + C::COL_DK;
       const uint32_t lk = lo_kmaj(sK), lv = lo_kmaj(sV), lk_mn = lo_mnmaj(sK);
-      const uint32_t lds_k = lo_kmaj(sDS), lds_mn = lo_mnmaj(sDS);
+      const uint32_t lds_mn = lo_mnmaj(sDS);
       auto wait_all = [&](uint32_t bar, uint32_t parity) {
         return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
       };
@@ -281,9 +282,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         if (!(ok = wait_all(bar_ds_ready, pi))) break;
         tc_fence_after_sync();
         if (elect_one()) {
+          // dS^T pairs sit in the dP columns like P^T in the S columns; dQ(i), issued after,
+          // overwrites them (d = 128) only once dK(i) has read them.
 #pragma unroll
           for (int kk = 0; kk < BWD_TILE / 16; ++kk)
-            mma_bf16_ss(tDK, desc(lds_k + koff(kk)), desc(lq_mn + mnoff(kk)), C::IDESC_KMN,
+            mma_bf16_ts(tDK, tDP + kk * 8 + (kk >= 4 ? 32 : 0), desc(lq_mn + mnoff(kk)), C::IDESC_KMN,
                         (i > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < BWD_TILE / 16; ++kk)
@@ -420,23 +423,28 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       RA_REG_FENCE32(dr);
       RA_REG_FENCE32((dr + 32));
       if (i > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(bar_ds_free, pi ^ 1u, abort_flag)))) return false;
-      // dS^T row (this key) x 64 queries -> 8 chunks of 16 B, chunk ch at slot ch ^ (row % 8).
+      // dS^T row (this key) x 64 queries: bf16 pairs into the dP columns just read (A of dK)
+      // and into shared memory, 8 chunks of 16 B, chunk ch at slot ch ^ (row % 8) (A of dQ).
+      uint32_t dsk[32];
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
         const float4 D0 = *reinterpret_cast<const float4*>(dls + 8 * ch);
         const float4 D1 = *reinterpret_cast<const float4*>(dls + 8 * ch + 4);
         const float dd[8] = {D0.x, D0.y, D0.z, D0.w, D1.x, D1.y, D1.z, D1.w};
-        uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int j0 = 8 * ch + 2 * e;
           const float a = p[j0] * (__uint_as_float(dr[j0]) - dd[2 * e]) * scale;
           const float b = p[j0 + 1] * (__uint_as_float(dr[j0 + 1]) - dd[2 * e + 1]) * scale;
-          w[e] = pack_bf16x2(a, b);
+          dsk[4 * ch + e] = pack_bf16x2(a, b);
         }
-        *reinterpret_cast<uint4*>(ds_row + ((ch ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(ds_row + ((ch ^ (row & 7)) << 4)) =
+            make_uint4(dsk[4 * ch], dsk[4 * ch + 1], dsk[4 * ch + 2], dsk[4 * ch + 3]);
       }
+      RA_TMEM_ST32(tDP + c0, dsk);
+      tmem_wait_st();
       fence_proxy_async_smem();
+      tc_fence_before_sync();
       mbar_arrive(bar_ds_ready);
       prev_qs = qs;
       prev_i0 = i0;
