@@ -1,6 +1,5 @@
 // bwd.cuh -- backward pass of ring attention: the problem plan, the key-tile / query-tile
-// walk, the row term D, the fp32 -> bf16 conversion of the dQ accumulator and the fp32
-// CUDA-core backward kernels.
+// walk, the row term D, helpers of the tensor-core kernels and the fp32 CUDA-core kernels.
 //
 // Gradients of O = softmax(S) V with S = Q K^T * scale ([BLOG] ring_attention_backward):
 //   P = exp(S - lse)            recomputed from the forward's log-sum-exp, no max pass
@@ -27,7 +26,7 @@ struct BwdPlan {
   const void* d_o;
   const float* lse;     // [BH, q_rows] natural-log lse of the forward
   const float* delta;   // [BH, q_rows] D = rowsum(dO * O)
-  float* dq;            // [BH, q_rows, d] fp32 (accumulated with atomics by the tensor-core kernel)
+  void* dq;             // [BH, q_rows, d]
   void* dk;             // [BH, k_rows, d]
   void* dv;             // [BH, k_rows, d]
   int BH;
@@ -35,8 +34,7 @@ struct BwdPlan {
   int P;
   int layout;
   int causal;
-  int accumulate;       // 1: dq, dk, dv are fp32 accumulators (+=); 0: written
-  int dkdv_bf16;        // 1: dk, dv written as bf16 (tensor-core kernel, accumulate == 0)
+  int accumulate;       // 1: dq, dk, dv are fp32 accumulators (+=); 0: written in the input dtype
   int64_t q_rows, k_rows, q_seg_len, k_seg_len;
   int64_t q_tok0, q_tok_stride, k_tok0, k_tok_stride;
   float scale;
@@ -111,15 +109,14 @@ __device__ __forceinline__ void walk_q_tiles(const BwdPlan& pl, const KTile& kt,
 }
 
 // ------------------------------------------------------------------------------------
-// D_i = sum_e dO_ie O_ie, one group of 8 lanes per row; optionally zeroes row i of an fp32
-// [rows, d] accumulator in the same pass.
+// D_i = sum_e dO_ie O_ie, one group of 8 lanes per row.
 // ------------------------------------------------------------------------------------
 constexpr int DELTA_THREADS = 256;
 
 template <bool BF16>
 __global__ void __launch_bounds__(DELTA_THREADS)
 bwd_delta_kernel(const void* __restrict__ o, const void* __restrict__ d_o, int64_t rows, int d,
-                 float* __restrict__ delta, float* __restrict__ zero_rows) {
+                 float* __restrict__ delta) {
   const int g = threadIdx.x & 7;
   const int64_t groups = (int64_t)gridDim.x * (DELTA_THREADS / 8);
   for (int64_t r = (int64_t)blockIdx.x * (DELTA_THREADS / 8) + (threadIdx.x >> 3); r < rows; r += groups) {
@@ -148,22 +145,112 @@ bwd_delta_kernel(const void* __restrict__ o, const void* __restrict__ d_o, int64
     acc += __shfl_xor_sync(0xffffffffu, acc, 2);
     acc += __shfl_xor_sync(0xffffffffu, acc, 4);
     if (g == 0) delta[r] = acc;
-    if (zero_rows != nullptr) {
-      float4* z = reinterpret_cast<float4*>(zero_rows + r * d);  // d % 4 == 0 here
-      for (int c = g; c < d / 4; c += 8) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
   }
 }
 
-// out[i] = bf16(acc[i]), n a multiple of 4.
-__global__ void __launch_bounds__(256)
-f32_to_bf16_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ out, int64_t n4) {
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
-    const float4 x = __ldcs(reinterpret_cast<const float4*>(acc) + i);
-    uint2 w;
-    w.x = pack_bf16x2(x.x, x.y);
-    w.y = pack_bf16x2(x.z, x.w);
-    reinterpret_cast<uint2*>(out)[i] = w;
+// ------------------------------------------------------------------------------------
+// Helpers of the tensor-core backward kernels (one thread = one TMEM lane, 64 columns).
+// ------------------------------------------------------------------------------------
+
+// p[j] = exp2(s_j * sl2 + nl2_j) for the 64 fp32 TMEM columns at taddr, where nl2_j is
+// -lse_j log2(e): nl2col[j] (a per-column value in shared memory) when PER_COL, else nl2row.
+// With `masked` (warp-uniform), columns outside [lo, hi) are 0. Paired f32x2 FMAs form the
+// exponents; MUFU ex2 evaluates them.
+template <bool PER_COL>
+__device__ __forceinline__ void bwd_exp_row64(uint32_t taddr, const float* nl2col, float nl2row, float sl2, bool masked,
+                                              int lo, int hi, float (&p)[64]) {
+  uint32_t sr[64];
+  RA_TMEM_LD32(taddr, sr);
+  RA_TMEM_LD32(taddr + 32, (sr + 32));
+  tmem_wait_ld();
+  RA_REG_FENCE32(sr);
+  RA_REG_FENCE32((sr + 32));
+  const uint64_t sl2x2 = f2_pack(sl2, sl2);
+#pragma unroll
+  for (int j = 0; j < 64; j += 4) {
+    float4 L = make_float4(nl2row, nl2row, nl2row, nl2row);
+    if (PER_COL) L = *reinterpret_cast<const float4*>(nl2col + j);
+    float x0, x1, x2, x3;
+    f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), sl2x2, f2_pack(L.x, L.y)), x0, x1);
+    f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3])), sl2x2, f2_pack(L.z, L.w)), x2,
+              x3);
+    p[j + 0] = ex2_approx(x0);
+    p[j + 1] = ex2_approx(x1);
+    p[j + 2] = ex2_approx(x2);
+    p[j + 3] = ex2_approx(x3);
+  }
+  if (masked) {
+#pragma unroll
+    for (int j = 0; j < 64; ++j) p[j] = (j >= lo && j < hi) ? p[j] : 0.f;
+  }
+}
+
+// ds = bf16 pairs of p_j (dP_j scale + nds_j) = p_j (dP_j - D_j) scale for the 64 fp32 dP
+// columns at taddr; nds_j = -D_j scale is ndscol[j] (per column, shared memory) when PER_COL,
+// else ndsrow. Two paired f32x2 operations per two scores.
+template <bool PER_COL>
+__device__ __forceinline__ void bwd_ds_row64(uint32_t taddr, const float (&p)[64], const float* ndscol, float ndsrow,
+                                             float scale, uint32_t (&ds)[32]) {
+  uint32_t dr[64];
+  RA_TMEM_LD32(taddr, dr);
+  RA_TMEM_LD32(taddr + 32, (dr + 32));
+  tmem_wait_ld();
+  RA_REG_FENCE32(dr);
+  RA_REG_FENCE32((dr + 32));
+  const uint64_t sc2 = f2_pack(scale, scale), z2 = f2_pack(0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < 64; j += 4) {
+    float4 N = make_float4(ndsrow, ndsrow, ndsrow, ndsrow);
+    if (PER_COL) N = *reinterpret_cast<const float4*>(ndscol + j);
+    const uint64_t t01 = f2_fma(f2_pack(__uint_as_float(dr[j]), __uint_as_float(dr[j + 1])), sc2, f2_pack(N.x, N.y));
+    const uint64_t t23 =
+        f2_fma(f2_pack(__uint_as_float(dr[j + 2]), __uint_as_float(dr[j + 3])), sc2, f2_pack(N.z, N.w));
+    float a, b, c, d;
+    f2_unpack(f2_fma(f2_pack(p[j], p[j + 1]), t01, z2), a, b);
+    f2_unpack(f2_fma(f2_pack(p[j + 2], p[j + 3]), t23, z2), c, d);
+    ds[j / 2] = pack_bf16x2(a, b);
+    ds[j / 2 + 1] = pack_bf16x2(c, d);
+  }
+}
+
+// Epilogue of an fp32 TMEM accumulator row: NC columns at taddr (all lanes of the warp load;
+// `have` false means the accumulator was never written and reads as 0). Valid rows are
+// written to dst + off as bf16, or added to the fp32 values there when `accumulate`.
+template <int NC>
+__device__ __forceinline__ void bwd_store_acc_row(uint32_t taddr, bool have, bool valid, void* dst, int64_t off,
+                                                  bool accumulate) {
+#pragma unroll
+  for (int cc = 0; cc < NC / 32; ++cc) {
+    uint32_t r[32];
+    if (have) {
+      RA_TMEM_LD32(taddr + cc * 32, r);
+      tmem_wait_ld();
+      RA_REG_FENCE32(r);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) r[j] = 0u;
+    }
+    if (!valid) continue;
+    if (accumulate) {
+      float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(dst) + off + cc * 32);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float4 a = o4[j];
+        a.x += __uint_as_float(r[4 * j]);
+        a.y += __uint_as_float(r[4 * j + 1]);
+        a.z += __uint_as_float(r[4 * j + 2]);
+        a.w += __uint_as_float(r[4 * j + 3]);
+        o4[j] = a;
+      }
+    } else {
+      uint4* o16 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + off + cc * 32);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        o16[j] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * j]), __uint_as_float(r[8 * j + 1])),
+                            pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3])),
+                            pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5])),
+                            pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7])));
+    }
   }
 }
 
@@ -339,7 +426,7 @@ bwd_dq_simt_f32_kernel(const BwdPlan pl, int64_t rows_per_pos) {
       }
     }
   }
-  float* dqp = pl.dq + ((int64_t)bh * pl.q_rows + qrow) * d;
+  float* dqp = static_cast<float*>(pl.dq) + ((int64_t)bh * pl.q_rows + qrow) * d;
 #pragma unroll
   for (int t = 0; t < SIMT_DMAX / 32; ++t) {
     const int e = lane + 32 * t;

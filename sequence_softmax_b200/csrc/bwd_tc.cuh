@@ -1,38 +1,41 @@
-// bwd_tc.cuh -- bf16 ring-attention backward on the 5th-generation tensor cores (sm_100a).
+// bwd_tc.cuh -- bf16 ring-attention backward, dK and dV, on the 5th-generation tensor cores
+// (sm_100a).
 //
 // Key-stationary: one CTA owns a tile of 128 keys of one virtual ring position and walks
 // every 128-row query tile that can see it, in ring order (positions c, c + 1, ... as the
 // KV chunk travels; see bwd.cuh). Its dK and dV stay in tensor memory for the whole walk
 // and are written once at the end, which is the "sum at the chunk's owner" of the ring
-// backward; dQ of each query tile is added to an fp32 accumulator in global memory with
-// vector reductions, staged through shared memory so that each instruction covers whole
-// 128-byte lines.
+// backward. dQ is computed by the query-stationary kernel of bwd_dq_tc.cuh, so no CTA adds
+// into memory another CTA writes: dQ, dK and dV are each produced by exactly one CTA and
+// the gradients are bitwise reproducible. (Adding each tile's dQ into a shared fp32
+// accumulator instead would cost 64 KB of global reductions per tile pair; measured on B200,
+// the L2 absorbs about 6 TB/s of fp32 reductions, ~21 B per clock per SM, which made that
+// traffic alone as long as the tile's five GEMMs.)
 //
 // Per query tile i (Q_i, dO_i, lse_i, D_i staged by TMA / the producer warp):
 //   S^T  = K Q_i^T             (M = keys, N = queries, K = d; both operands K-major)
 //   dP^T = V dO_i^T            (same form)
 //   P^T  = exp2(S^T scale log2e - lse_i log2e), masked; bf16 into the S columns of TMEM
 //   dV  += P^T dO_i            (A = P^T from TMEM, B = dO_i MN-major)
-//   dS^T = P^T (dP^T - D_i) scale, bf16 into the dP columns of TMEM and into a
-//                              128B-swizzled shared-memory tile
+//   dS^T = P^T (dP^T - D_i) scale, bf16 into the dP columns of TMEM
 //   dK  += dS^T Q_i            (A = dS^T from TMEM, B = Q_i MN-major)
-//   dQ_i = dS K                (A = the same dS tile read MN-major, B = K MN-major)
-// so each (query tile, key tile) pair costs five 128 x 128 x d GEMMs and one exponential per
-// score, and P and dS never leave the SM.
+// Four 128 x 128 x d GEMMs and one exponential per score; P and dS never leave the SM.
 //
 // Warp roles (384 threads, 3 warpgroups; setmaxnreg moves registers to the math warps):
 //   warps 0-3, 4-7  math: thread t of warpgroup g owns key row t (TMEM lane t) and query
-//                   columns 64g .. 64g + 63 of S^T / dP^T; for dQ it owns query row t and
-//                   columns g d/2 .. g d/2 + d/2 - 1
-//   warp 8          producer: K and V once, then Q_i and dO_i by TMA into a 2-stage ring,
-//                   with lse_i log2e and D_i stored beside them
-//   warp 9          MMA issuer (the whole warp loops, one elected lane issues)
+//                   columns 64g .. 64g + 63 of S^T / dP^T, and dK / dV columns
+//                   g d/2 .. g d/2 + d/2 - 1 in the epilogue
+//   warp 8          producer: K and V once, then Q_i (3 stages) and dO_i (2 stages) by TMA,
+//                   and -lse_i log2e, -D_i scale (read a tile ahead) into a 2-slot ring
+//   warp 9          MMA issuer (the whole warp loops, one elected lane issues); order per
+//                   tile: dP(i), dV(i), S(i+1), dK(i), so that P(i+1) is computed while
+//                   dK(i) runs
 //
-// Tensor memory (512 columns): S^T/P^T [0,128) | dP^T [128,256) | dV | dK, with dQ_i in the
-// dP^T columns for d = 128 (issued after the math warps have read dP^T; the next dP^T waits
-// until dQ_i has been read) and in free columns [256, 320) for d = 64.
+// Tensor memory (512 columns at d = 128): S^T/P^T [0,128) | dP^T/dS^T [128,256) | dV | dK.
+// MMAs issued by one thread execute in order, so S(i+1) overwrites P(i) only after dV(i)
+// has read it, and dP(i+1) overwrites dS(i) only after dK(i) has read it.
 //
-// Query rows beyond a segment's end get lse log2e = +inf and D = 0, so their P and dS are
+// Query rows beyond a segment's end get -lse log2e = -inf and D = 0, so their P and dS are
 // exactly 0 and they add nothing to dK, dV; key rows beyond the end get P = dS = 0 and are
 // not written. A query row whose forward lse is -inf saw no key and gets P = 0 as well.
 #pragma once
@@ -46,19 +49,7 @@ constexpr int BW_WARP_PRODUCER = 8;
 constexpr int BW_WARP_MMA = 9;
 constexpr int BW_REGS_MATH = 216;   // 2 x 216 + 72 = 504 = 168 * 384 / 128
 constexpr int BW_REGS_OTHER = 72;
-constexpr int BW_NSTAGE = 2;
 constexpr int BW_TMEM_COLS = 512;
-
-// Barrier among the `n` threads that use named barrier `id` (0 is __syncthreads).
-__device__ __forceinline__ void named_bar_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
-// Fire-and-forget vector reduction into global memory (no value returned, so no wait).
-__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
-  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
 
 template <int D>
 struct BwCfg {
@@ -66,36 +57,33 @@ struct BwCfg {
   static constexpr int BOX_BYTES = BWD_TILE * 64 * 2;       // one TMA box: 128 rows x 64 bf16
   static constexpr int NBOX = D / 64;
   static constexpr int TILE_BYTES = NBOX * BOX_BYTES;       // a K, V, Q or dO tile
-  static constexpr int DS_BYTES = 2 * BOX_BYTES;            // dS^T: 128 keys x 128 queries
+  // Q feeds S(i+1), which is issued before dK(i) frees Q(i): three Q stages give its load two
+  // tiles of lead. dO is last read by dV, earlier in the tile: two stages suffice.
+  static constexpr int NQ = (D == 128) ? 3 : 4;
+  static constexpr int NDO = (D == 128) ? 2 : 4;
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = TILE_BYTES;
-  static constexpr int Q_OFF = 2 * TILE_BYTES;              // stage s: Q at +2s TILE, dO at +(2s+1) TILE
-  static constexpr int DS_OFF = Q_OFF + BW_NSTAGE * 2 * TILE_BYTES;
-  static constexpr int LD_OFF = DS_OFF + DS_BYTES;          // stage s: lse log2e [128], D [128]
-  static constexpr int BAR_OFF = LD_OFF + BW_NSTAGE * 2 * BWD_TILE * 4;
-  static constexpr int NBAR = 16;
+  static constexpr int Q_OFF = 2 * TILE_BYTES;
+  static constexpr int DO_OFF = Q_OFF + NQ * TILE_BYTES;
+  static constexpr int LD_OFF = DO_OFF + NDO * TILE_BYTES;  // slot s: -lse log2e [128], -D scale [128]
+  static constexpr int BAR_OFF = LD_OFF + 2 * 2 * BWD_TILE * 4;
+  static constexpr int NBAR = 1 + 2 * NQ + 2 * NDO + 4 + 6;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16;
-  static constexpr int COL_S = 0, COL_DP = 128;
-  static constexpr int COL_DQ = (D == 128) ? 128 : 256;
-  static constexpr int COL_DV = (D == 128) ? 256 : 320;
-  static constexpr int COL_DK = COL_DV + D;
-  static constexpr bool DQ_IN_DP = D == 128;
+  static constexpr int COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
   static constexpr uint32_t IDESC_SS = idesc_bf16_f32_ab(128, 128, false, false);
   static constexpr uint32_t IDESC_KMN = idesc_bf16_f32_ab(128, D, false, true);  // dV, dK
-  static constexpr uint32_t IDESC_DQ = idesc_bf16_f32_ab(128, D, true, true);
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
   static_assert(COL_DK + D <= BW_TMEM_COLS, "tensor memory columns");
 };
 
 template <int D>
 __global__ void __launch_bounds__(BW_THREADS, 1)
-attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                   const BwdPlan pl) {
+attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                        const BwdPlan pl) {
   using C = BwCfg<D>;
-  // The 128-byte swizzle needs 1 KB-aligned tiles; the whole budget is used, so there is
-  // no slack to align by hand: the declaration asks for it and the kernel checks it.
+  // 128-byte-swizzled tiles need 1 KB alignment: asked of the declaration, checked here.
   extern __shared__ __align__(1024) uint8_t bw_smem[];
   uint8_t* smem = bw_smem;
   const uint32_t sbase = smem_u32(smem);
@@ -103,16 +91,20 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (threadIdx.x == 0) record_error(DEVERR_BOUNDS);
     return;
   }
-  const uint32_t sK = sbase + C::K_OFF, sV = sbase + C::V_OFF, sDS = sbase + C::DS_OFF;
-  auto sQ = [&](int st) { return sbase + C::Q_OFF + (uint32_t)(2 * st) * C::TILE_BYTES; };
-  auto sDO = [&](int st) { return sbase + C::Q_OFF + (uint32_t)(2 * st + 1) * C::TILE_BYTES; };
+  const uint32_t sK = sbase + C::K_OFF, sV = sbase + C::V_OFF;
+  auto sQ = [&](int st) { return sbase + C::Q_OFF + (uint32_t)st * C::TILE_BYTES; };
+  auto sDO = [&](int st) { return sbase + C::DO_OFF + (uint32_t)st * C::TILE_BYTES; };
   const uint32_t bar0 = sbase + C::BAR_OFF;
   const uint32_t bar_kv_full = bar0;
   auto bar_q_full = [&](int st) { return bar0 + 8u * (1 + st); };
-  auto bar_q_empty = [&](int st) { return bar0 + 8u * (3 + st); };
-  const uint32_t bar_s_full = bar0 + 8u * 5, bar_dp_full = bar0 + 8u * 6, bar_p_ready = bar0 + 8u * 7,
-                 bar_ds_ready = bar0 + 8u * 8, bar_ds_free = bar0 + 8u * 9, bar_dq_full = bar0 + 8u * 10,
-                 bar_dq_free = bar0 + 8u * 11, bar_acc_done = bar0 + 8u * 12, bar_drain = bar0 + 8u * 13;
+  auto bar_q_empty = [&](int st) { return bar0 + 8u * (1 + C::NQ + st); };
+  auto bar_do_full = [&](int st) { return bar0 + 8u * (1 + 2 * C::NQ + st); };
+  auto bar_do_empty = [&](int st) { return bar0 + 8u * (1 + 2 * C::NQ + C::NDO + st); };
+  auto bar_ld_full = [&](int sl) { return bar0 + 8u * (1 + 2 * C::NQ + 2 * C::NDO + sl); };
+  auto bar_ld_empty = [&](int sl) { return bar0 + 8u * (3 + 2 * C::NQ + 2 * C::NDO + sl); };
+  const uint32_t bar_s_full = bar0 + 8u * (5 + 2 * C::NQ + 2 * C::NDO), bar_dp_full = bar_s_full + 8u,
+                 bar_p_ready = bar_s_full + 16u, bar_ds_ready = bar_s_full + 24u, bar_acc_done = bar_s_full + 32u,
+                 bar_drain = bar_s_full + 40u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
 
@@ -125,17 +117,22 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
   if (threadIdx.x == 0) {
     mbar_init(bar_kv_full, 1);
-    for (int st = 0; st < BW_NSTAGE; ++st) {
-      mbar_init(bar_q_full(st), 1 + 32);  // TMA transaction arrive + the producer's 32 lanes
+    for (int st = 0; st < C::NQ; ++st) {
+      mbar_init(bar_q_full(st), 1);
       mbar_init(bar_q_empty(st), 1);
+    }
+    for (int st = 0; st < C::NDO; ++st) {
+      mbar_init(bar_do_full(st), 1);
+      mbar_init(bar_do_empty(st), 1);
+    }
+    for (int sl = 0; sl < 2; ++sl) {
+      mbar_init(bar_ld_full(sl), 32);    // the producer's 32 lanes
+      mbar_init(bar_ld_empty(sl), 256);  // every math thread, done with the slot
     }
     mbar_init(bar_s_full, 1);
     mbar_init(bar_dp_full, 1);
     mbar_init(bar_p_ready, 256);
     mbar_init(bar_ds_ready, 256);
-    mbar_init(bar_ds_free, 1);
-    mbar_init(bar_dq_full, 1);
-    mbar_init(bar_dq_free, 256);
     mbar_init(bar_acc_done, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -172,43 +169,72 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           tma_load_4d(sV + b * C::BOX_BYTES, &tm_v, bar_kv_full, 64 * b, ky, kz, bh);
         }
       }
+      // lse / D of a tile are read from global memory one tile ahead into registers and
+      // stored into their slot when the next tile is issued, so their latency is hidden.
+      // The loads are unconditional (rows past the segment end read a valid row and are
+      // overridden at store time), so nothing waits for them before the store.
+      float ld_l[BWD_TILE / 32], ld_d[BWD_TILE / 32];
+      uint32_t ld_valid = 0;
+      auto load_ld = [&](const Seg& qs, int64_t i0) {
+        ld_valid = 0;
+#pragma unroll
+        for (int m = 0; m < BWD_TILE / 32; ++m) {
+          const int64_t li = i0 + lane + 32 * m;
+          const bool v = li < qs.count;
+          ld_valid |= (v ? 1u : 0u) << m;
+          const int64_t idx = (int64_t)bh * pl.q_rows + qs.row0 + qs.stride * (v ? li : 0);
+          ld_l[m] = pl.lse[idx];
+          ld_d[m] = pl.delta[idx];
+        }
+      };
+      auto store_ld = [&](int u) {  // tile u's values into slot u & 1
+        const int sl = u & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_ld_empty(sl), ((uint32_t)(u >> 1) & 1u) ^ 1u, abort_flag)))
+          return false;
+        float* l2s = reinterpret_cast<float*>(smem + C::LD_OFF + sl * 2 * BWD_TILE * 4);
+#pragma unroll
+        for (int m = 0; m < BWD_TILE / 32; ++m) {
+          // rows past the segment end, or that saw no key in the forward: P = 0 and dS = 0
+          const bool v = (ld_valid >> m) & 1u;
+          l2s[lane + 32 * m] = (v && ld_l[m] != -INFINITY) ? -ld_l[m] * 1.4426950408889634f : -INFINITY;
+          l2s[BWD_TILE + lane + 32 * m] = v ? -ld_d[m] * pl.scale : 0.f;
+        }
+        mbar_arrive(bar_ld_full(sl));
+        return true;
+      };
       int issued = 0;
       walk_q_tiles(pl, kt, [&](const Seg& qs, int64_t i0) {
-        const int st = issued & 1;
-        const uint32_t ph = (uint32_t)(issued >> 1) & 1u;
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_q_empty(st), ph ^ 1u, abort_flag))) return false;
+        const int i = issued;
+        if (i > 0 && !store_ld(i - 1)) return false;
+        const int sq = i % C::NQ, sd = i % C::NDO;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_q_empty(sq), ((uint32_t)(i / C::NQ) & 1u) ^ 1u, abort_flag)))
+          return false;
+        const int qy = (int)(qs.row0 % qs.stride);
+        const int qz = (int)(qs.row0 / qs.stride + i0);
         if (lane == 0) {
-          mbar_arrive_expect_tx(bar_q_full(st), 2 * C::TILE_BYTES);
-          const int qy = (int)(qs.row0 % qs.stride);
-          const int qz = (int)(qs.row0 / qs.stride + i0);
-          for (int b = 0; b < C::NBOX; ++b) {
-            tma_load_4d(sQ(st) + b * C::BOX_BYTES, &tm_q, bar_q_full(st), 64 * b, qy, qz, bh);
-            tma_load_4d(sDO(st) + b * C::BOX_BYTES, &tm_do, bar_q_full(st), 64 * b, qy, qz, bh);
-          }
+          mbar_arrive_expect_tx(bar_q_full(sq), C::TILE_BYTES);
+          for (int b = 0; b < C::NBOX; ++b)
+            tma_load_4d(sQ(sq) + b * C::BOX_BYTES, &tm_q, bar_q_full(sq), 64 * b, qy, qz, bh);
         }
-        float* l2s = reinterpret_cast<float*>(smem + C::LD_OFF + st * 2 * BWD_TILE * 4);
-        float* dls = l2s + BWD_TILE;
-        for (int r = lane; r < BWD_TILE; r += 32) {
-          const int64_t li = i0 + r;
-          float l2 = INFINITY, dd = 0.f;
-          if (li < qs.count) {
-            const int64_t idx = (int64_t)bh * pl.q_rows + qs.row0 + qs.stride * li;
-            const float l = pl.lse[idx];
-            if (l != -INFINITY) l2 = l * 1.4426950408889634f;
-            dd = pl.delta[idx];
-          }
-          l2s[r] = l2;
-          dls[r] = dd;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_do_empty(sd), ((uint32_t)(i / C::NDO) & 1u) ^ 1u, abort_flag)))
+          return false;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar_do_full(sd), C::TILE_BYTES);
+          for (int b = 0; b < C::NBOX; ++b)
+            tma_load_4d(sDO(sd) + b * C::BOX_BYTES, &tm_do, bar_do_full(sd), 64 * b, qy, qz, bh);
         }
-        mbar_arrive(bar_q_full(st));
+        load_ld(qs, i0);
         ++issued;
         return true;
       });
+      if (issued == T) store_ld(T - 1);
       // Drain: every TMA load issued lands before the CTA's shared memory goes away.
       if (lane == 0) {
         mbar_wait_drain(bar_kv_full, 0);
-        for (int u = issued > BW_NSTAGE ? issued - BW_NSTAGE : 0; u < issued; ++u)
-          mbar_wait_drain(bar_q_full(u & 1), (uint32_t)(u >> 1) & 1u);
+        for (int u = issued > C::NQ ? issued - C::NQ : 0; u < issued; ++u)
+          mbar_wait_drain(bar_q_full(u % C::NQ), (uint32_t)(u / C::NQ) & 1u);
+        for (int u = issued > C::NDO ? issued - C::NDO : 0; u < issued; ++u)
+          mbar_wait_drain(bar_do_full(u % C::NDO), (uint32_t)(u / C::NDO) & 1u);
       }
       __syncwarp();
     }
@@ -223,10 +249,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       auto koff = [](int kk) { return (uint32_t)(((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4); };
       // MN-major k-step: 16 rows of 128 B.
       auto mnoff = [](int kk) { return (uint32_t)(kk * (2048 >> 4)); };
-      const uint32_t tS = tmem + C::COL_S, tDP = tmem + C::COL_DP, tDQ = tmem + C::COL_DQ,
-                     tDV = tmem + C::COL_DV, tDK = tmem + C::COL_DK;
-      const uint32_t lk = lo_kmaj(sK), lv = lo_kmaj(sV), lk_mn = lo_mnmaj(sK);
-      const uint32_t lds_mn = lo_mnmaj(sDS);
+      const uint32_t tS = tmem + C::COL_S, tDP = tmem + C::COL_DP, tDV = tmem + C::COL_DV, tDK = tmem + C::COL_DK;
+      const uint32_t lk = lo_kmaj(sK), lv = lo_kmaj(sV);
       auto wait_all = [&](uint32_t bar, uint32_t parity) {
         return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
       };
@@ -237,8 +261,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           mma_bf16_ss(tS, desc(lk + koff(kk)), desc(lq + koff(kk)), C::IDESC_SS, kk > 0);
         tc_commit(bar_s_full);
       };
-      // Order per query tile i: dP(i), dV(i), S(i+1), dK(i), dQ(i). S(i+1) goes ahead of
-      // dK(i) and dQ(i) so that the math warps can exponentiate tile i + 1 while those run.
       bool ok = wait_all(bar_kv_full, 0) && wait_all(bar_q_full(0), 0);
       if (ok) {
         tc_fence_after_sync();
@@ -246,14 +268,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         __syncwarp();
       }
       for (int i = 0; i < T && ok; ++i) {
-        const int st = i & 1;
+        const int sq = i % C::NQ, sd = i % C::NDO;
         const uint32_t pi = (uint32_t)i & 1u;
-        const uint32_t ldo = lo_kmaj(sDO(st)), lq_mn = lo_mnmaj(sQ(st)), ldo_mn = lo_mnmaj(sDO(st));
-        if (C::DQ_IN_DP && i > 0) {
-          // dQ(i-1) occupies the dP columns until the math warps have read it.
-          if (!(ok = wait_all(bar_dq_free, pi ^ 1u))) break;
-          tc_fence_after_sync();
-        }
+        const uint32_t ldo = lo_kmaj(sDO(sd)), lq_mn = lo_mnmaj(sQ(sq)), ldo_mn = lo_mnmaj(sDO(sd));
+        if (!(ok = wait_all(bar_do_full(sd), (uint32_t)(i / C::NDO) & 1u))) break;
+        tc_fence_after_sync();
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
@@ -269,31 +288,26 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           for (int kk = 0; kk < BWD_TILE / 16; ++kk)
             mma_bf16_ts(tDV, tS + kk * 8 + (kk >= 4 ? 32 : 0), desc(ldo_mn + mnoff(kk)), C::IDESC_KMN,
                         (i > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bar_do_empty(sd));  // dO(i) is last read by dV(i)
         }
         __syncwarp();
         if (i + 1 < T) {
           // S(i+1) overwrites the S columns only after dV(i) (issued above) has read P(i).
-          const int st1 = (i + 1) & 1;
-          if (!(ok = wait_all(bar_q_full(st1), (uint32_t)((i + 1) >> 1) & 1u))) break;
+          const int sq1 = (i + 1) % C::NQ;
+          if (!(ok = wait_all(bar_q_full(sq1), (uint32_t)((i + 1) / C::NQ) & 1u))) break;
           tc_fence_after_sync();
-          if (elect_one()) issue_s(st1);
+          if (elect_one()) issue_s(sq1);
           __syncwarp();
         }
         if (!(ok = wait_all(bar_ds_ready, pi))) break;
         tc_fence_after_sync();
         if (elect_one()) {
-          // dS^T pairs sit in the dP columns like P^T in the S columns; dQ(i), issued after,
-          // overwrites them (d = 128) only once dK(i) has read them.
+          // dS^T pairs sit in the dP columns like P^T in the S columns.
 #pragma unroll
           for (int kk = 0; kk < BWD_TILE / 16; ++kk)
             mma_bf16_ts(tDK, tDP + kk * 8 + (kk >= 4 ? 32 : 0), desc(lq_mn + mnoff(kk)), C::IDESC_KMN,
                         (i > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < BWD_TILE / 16; ++kk)
-            mma_bf16_ss(tDQ, desc(lds_mn + mnoff(kk)), desc(lk_mn + mnoff(kk)), C::IDESC_DQ, kk > 0);
-          tc_commit(bar_dq_full);
-          tc_commit(bar_ds_free);
-          tc_commit(bar_q_empty(st));
+          tc_commit(bar_q_empty(sq));  // Q(i) is last read by dK(i)
           if (i == T - 1) tc_commit(bar_acc_done);
         }
         __syncwarp();
@@ -311,60 +325,14 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int row = threadIdx.x & 127;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const int c0 = 64 * g;  // this thread's query columns of S^T / dP^T
-    const uint32_t tS = tmem + C::COL_S + lane_off, tDP = tmem + C::COL_DP + lane_off,
-                   tDQ = tmem + C::COL_DQ + lane_off;
+    const uint32_t tS = tmem + C::COL_S + lane_off, tDP = tmem + C::COL_DP + lane_off;
     const int64_t jl = kt.j0 + row;
     const bool kvalid = jl < kt.seg.count;
     const int64_t tk = pl.k_tok0 + pl.k_tok_stride * (kt.seg.row0 + kt.seg.stride * jl);
-    const float sl2 = pl.scale_log2, scale = pl.scale;
-    uint8_t* ds_row = smem + C::DS_OFF + g * C::BOX_BYTES + row * 128;
     int i = 0;
     bool ok = true;
-    Seg prev_qs{0, 1, 0};
-    int64_t prev_i0 = 0;
-    // dQ(j) of query tile j (i0 = its first local row): thread = query row `row`, columns
-    // g d/2 .. g d/2 + d/2 - 1. The values are read out of TMEM and the columns released first,
-    // so the next dP never waits on the reductions. The reductions go through this
-    // warpgroup's half of the dS tile (idle from dQ(j)'s completion until dS(j+1) is written)
-    // in rounds of 32 columns: each thread stores its row, then each warp reduces 4 rows x
-    // 128 contiguous bytes per vector instruction -- twice the L2 reduction throughput of one
-    // 16-byte piece of 32 different rows per instruction (measured on B200: 6.3 vs 3.1 TB/s).
-    auto flush_dq = [&](const Seg& qs, int64_t i0, uint32_t parity) -> bool {
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_dq_full, parity, abort_flag))) return false;
-      tc_fence_after_sync();
-      uint32_t r[D / 2];
-#pragma unroll
-      for (int cc = 0; cc < D / 64; ++cc) RA_TMEM_LD32(tDQ + g * (D / 2) + cc * 32, (r + 32 * cc));
-      tmem_wait_ld();
-#pragma unroll
-      for (int cc = 0; cc < D / 64; ++cc) RA_REG_FENCE32((r + 32 * cc));
-      tc_fence_before_sync();
-      mbar_arrive(bar_dq_free);
-      uint8_t* stg = smem + C::DS_OFF + g * C::BOX_BYTES;  // 128 rows x 128 B, 16-B chunks swizzled
-      const int wq = warp & 3;
-      const int64_t row_base = (int64_t)bh * pl.q_rows + qs.row0;
-#pragma unroll
-      for (int k = 0; k < D / 64; ++k) {
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(stg + row * 128 + ((c ^ (row & 7)) << 4)) =
-              make_uint4(r[32 * k + 4 * c], r[32 * k + 4 * c + 1], r[32 * k + 4 * c + 2], r[32 * k + 4 * c + 3]);
-        named_bar_sync(1 + g, 128);
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const int R = 32 * wq + 4 * m + (lane >> 3), c = lane & 7;
-          const float4 v = *reinterpret_cast<const float4*>(stg + R * 128 + ((c ^ (R & 7)) << 4));
-          const int64_t li = i0 + R;
-          if (li < qs.count)
-            red_add_v4(pl.dq + (row_base + qs.stride * li) * D + g * (D / 2) + 32 * k + 4 * c, v.x, v.y, v.z, v.w);
-        }
-        named_bar_sync(1 + g, 128);  // the next round (or dS) overwrites the staging rows
-      }
-      return true;
-    };
-    // Per query tile i: P(i), then dQ(i-1), then dS(i) (the MMA warp's order above).
     walk_q_tiles(pl, kt, [&](const Seg& qs, int64_t i0) {
-      const int st = i & 1;
+      const int sl = i & 1;
       const uint32_t ph = (uint32_t)(i >> 1) & 1u, pi = (uint32_t)i & 1u;
       // Causal: query column c (token tq0 + tqs c) sees this key iff c >= lo.
       const int64_t tqs = pl.q_tok_stride * qs.stride;
@@ -375,33 +343,15 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const int64_t cmin = (tk - tq0 + tqs - 1) / tqs;
         lo = cmin > BWD_TILE ? BWD_TILE : (int)cmin;
       }
-      const bool nomask = __all_sync(0xffffffffu, lo <= c0);
-      const float* l2s = reinterpret_cast<const float*>(smem + C::LD_OFF + st * 2 * BWD_TILE * 4) + c0;
+      // columns c0 .. c0 + 63 of this thread: those below `lo` are masked
+      const bool masked = !__all_sync(0xffffffffu, lo <= c0);
+      const float* l2s = reinterpret_cast<const float*>(smem + C::LD_OFF + sl * 2 * BWD_TILE * 4) + c0;
       const float* dls = l2s + BWD_TILE;
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar_q_full(st), ph, abort_flag)))) return false;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar_ld_full(sl), ph, abort_flag)))) return false;
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full, pi, abort_flag)))) return false;
       tc_fence_after_sync();
       float p[64];
-      {
-        uint32_t sr[64];
-        RA_TMEM_LD32(tS + c0, sr);
-        RA_TMEM_LD32(tS + c0 + 32, (sr + 32));
-        tmem_wait_ld();
-        RA_REG_FENCE32(sr);
-        RA_REG_FENCE32((sr + 32));
-#pragma unroll
-        for (int j = 0; j < 64; j += 4) {
-          const float4 L = *reinterpret_cast<const float4*>(l2s + j);
-          p[j + 0] = ex2_approx(fmaf(__uint_as_float(sr[j + 0]), sl2, -L.x));
-          p[j + 1] = ex2_approx(fmaf(__uint_as_float(sr[j + 1]), sl2, -L.y));
-          p[j + 2] = ex2_approx(fmaf(__uint_as_float(sr[j + 2]), sl2, -L.z));
-          p[j + 3] = ex2_approx(fmaf(__uint_as_float(sr[j + 3]), sl2, -L.w));
-        }
-      }
-      if (!nomask) {
-#pragma unroll
-        for (int j = 0; j < 64; ++j) p[j] = (c0 + j >= lo) ? p[j] : 0.f;
-      }
+      bwd_exp_row64<true>(tS + c0, l2s, 0.f, pl.scale_log2, masked, lo - c0, 64, p);
       {
         uint32_t pk[32];
 #pragma unroll
@@ -412,46 +362,19 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       tc_fence_before_sync();
       mbar_arrive(bar_p_ready);
 
-      if (i > 0 && !(ok = flush_dq(prev_qs, prev_i0, pi ^ 1u))) return false;
-
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_full, pi, abort_flag)))) return false;
       tc_fence_after_sync();
-      uint32_t dr[64];
-      RA_TMEM_LD32(tDP + c0, dr);
-      RA_TMEM_LD32(tDP + c0 + 32, (dr + 32));
-      tmem_wait_ld();
-      RA_REG_FENCE32(dr);
-      RA_REG_FENCE32((dr + 32));
-      if (i > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(bar_ds_free, pi ^ 1u, abort_flag)))) return false;
-      // dS^T row (this key) x 64 queries: bf16 pairs into the dP columns just read (A of dK)
-      // and into shared memory, 8 chunks of 16 B, chunk ch at slot ch ^ (row % 8) (A of dQ).
+      // dS^T row (this key) x 64 queries: bf16 pairs into the dP columns just read (A of dK).
       uint32_t dsk[32];
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const float4 D0 = *reinterpret_cast<const float4*>(dls + 8 * ch);
-        const float4 D1 = *reinterpret_cast<const float4*>(dls + 8 * ch + 4);
-        const float dd[8] = {D0.x, D0.y, D0.z, D0.w, D1.x, D1.y, D1.z, D1.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int j0 = 8 * ch + 2 * e;
-          const float a = p[j0] * (__uint_as_float(dr[j0]) - dd[2 * e]) * scale;
-          const float b = p[j0 + 1] * (__uint_as_float(dr[j0 + 1]) - dd[2 * e + 1]) * scale;
-          dsk[4 * ch + e] = pack_bf16x2(a, b);
-        }
-        *reinterpret_cast<uint4*>(ds_row + ((ch ^ (row & 7)) << 4)) =
-            make_uint4(dsk[4 * ch], dsk[4 * ch + 1], dsk[4 * ch + 2], dsk[4 * ch + 3]);
-      }
+      bwd_ds_row64<true>(tDP + c0, p, dls, 0.f, pl.scale, dsk);
       RA_TMEM_ST32(tDP + c0, dsk);
       tmem_wait_st();
-      fence_proxy_async_smem();
       tc_fence_before_sync();
       mbar_arrive(bar_ds_ready);
-      prev_qs = qs;
-      prev_i0 = i0;
+      mbar_arrive(bar_ld_empty(sl));  // done with this tile's -lse log2e and -D scale
       ++i;
       return true;
     });
-    if (ok && T > 0) ok = flush_dq(prev_qs, prev_i0, (uint32_t)(T - 1) & 1u);
 
     // ---- epilogue: dV and dK of this thread's key row, columns g d/2 .. g d/2 + d/2 - 1
     if (ok && T > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_acc_done, 0, abort_flag));
@@ -459,44 +382,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       if (T > 0) tc_fence_after_sync();
       const int64_t krow = kt.seg.row0 + kt.seg.stride * jl;
       const int64_t off = ((int64_t)bh * pl.k_rows + krow) * D + g * (D / 2);
-#pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const uint32_t tAcc = tmem + (m == 0 ? C::COL_DV : C::COL_DK) + lane_off + g * (D / 2);
-        void* dst = m == 0 ? pl.dv : pl.dk;
-#pragma unroll
-        for (int cc = 0; cc < D / 64; ++cc) {
-          uint32_t r[32];
-          if (T > 0) {
-            RA_TMEM_LD32(tAcc + cc * 32, r);
-            tmem_wait_ld();
-            RA_REG_FENCE32(r);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) r[j] = 0u;
-          }
-          if (!kvalid) continue;
-          if (pl.accumulate) {
-            float4* o4 = reinterpret_cast<float4*>(static_cast<float*>(dst) + off + cc * 32);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              float4 a = o4[j];
-              a.x += __uint_as_float(r[4 * j]);
-              a.y += __uint_as_float(r[4 * j + 1]);
-              a.z += __uint_as_float(r[4 * j + 2]);
-              a.w += __uint_as_float(r[4 * j + 3]);
-              o4[j] = a;
-            }
-          } else {
-            uint4* o16 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(dst) + off + cc * 32);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              o16[j] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * j]), __uint_as_float(r[8 * j + 1])),
-                                  pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3])),
-                                  pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5])),
-                                  pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7])));
-          }
-        }
-      }
+      bwd_store_acc_row<D / 2>(tmem + C::COL_DV + lane_off + g * (D / 2), T > 0, kvalid, pl.dv, off,
+                               pl.accumulate != 0);
+      bwd_store_acc_row<D / 2>(tmem + C::COL_DK + lane_off + g * (D / 2), T > 0, kvalid, pl.dk, off,
+                               pl.accumulate != 0);
     }
   }
 

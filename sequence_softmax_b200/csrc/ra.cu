@@ -10,6 +10,7 @@
 #include "merge.cuh"
 #include "bwd.cuh"
 #include "bwd_tc.cuh"
+#include "bwd_dq_tc.cuh"
 
 #define RA_ABI_VERSION 2
 
@@ -128,26 +129,31 @@ ra_status set_smem_attr_once(K* fn, int bytes, bool (&done)[64]) {
   return RA_OK;
 }
 
+// Both tensor-core gradient kernels of one plan: key-stationary dK/dV, then query-stationary dQ.
 template <int D>
 ra_status launch_bwd_tc(const BwdPlan& pl, int S, cudaStream_t stream) {
-  using C = BwCfg<D>;
   CUtensorMap mq, mk, mv, mdo;
   if (!make_tile_map(&mq, pl.q, pl.BH, pl.q_rows, D, S) || !make_tile_map(&mk, pl.k, pl.BH, pl.k_rows, D, S) ||
       !make_tile_map(&mv, pl.v, pl.BH, pl.k_rows, D, S) || !make_tile_map(&mdo, pl.d_o, pl.BH, pl.q_rows, D, S))
     return RA_ERR_CUDA;
-  static bool done[64] = {};
-  ra_status st = set_smem_attr_once(attn_bwd_tc_kernel<D>, C::SMEM_BYTES, done);
+  static bool done_kv[64] = {}, done_q[64] = {};
+  ra_status st = set_smem_attr_once(attn_bwd_dkdv_tc_kernel<D>, BwCfg<D>::SMEM_BYTES, done_kv);
   if (st != RA_OK) return st;
-  const int64_t nkt = (pl.k_seg_len + BWD_TILE - 1) / BWD_TILE;
-  const int64_t grid = nkt * (int64_t)pl.P * num_segments(pl.layout) * pl.BH;
-  if (grid <= 0) return RA_OK;
-  if (grid > 0x7FFFFFFFll) return RA_ERR_UNSUPPORTED;
-  attn_bwd_tc_kernel<D><<<(unsigned)grid, BW_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, pl);
+  st = set_smem_attr_once(attn_bwd_dq_tc_kernel<D>, BqCfg<D>::SMEM_BYTES, done_q);
+  if (st != RA_OK) return st;
+  const int64_t segs = (int64_t)pl.P * num_segments(pl.layout);
+  const int64_t grid_kv = (pl.k_seg_len + BWD_TILE - 1) / BWD_TILE * segs * pl.BH;
+  const int64_t grid_q = (pl.q_seg_len + BWD_TILE - 1) / BWD_TILE * segs * pl.BH;
+  if (grid_kv > 0x7FFFFFFFll || grid_q > 0x7FFFFFFFll) return RA_ERR_UNSUPPORTED;
+  if (grid_kv > 0)
+    attn_bwd_dkdv_tc_kernel<D><<<(unsigned)grid_kv, BW_THREADS, BwCfg<D>::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, pl);
+  if (grid_q > 0)
+    attn_bwd_dq_tc_kernel<D><<<(unsigned)grid_q, BQ_THREADS, BqCfg<D>::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, pl);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
-// The gradient kernels of one plan: the tensor-core kernel for bf16, the two fp32 kernels
-// otherwise. S = row spacing of the striped view (P) or 1.
+// The gradient kernels of one plan: the two tensor-core kernels for bf16, the two fp32
+// kernels otherwise. S = row spacing of the striped view (P) or 1.
 ra_status launch_backward(const BwdPlan& pl, ra_dtype dt, int S, cudaStream_t stream) {
   if (dt == RA_BF16) {
     if (pl.d == 128) return launch_bwd_tc<128>(pl, S, stream);
@@ -164,14 +170,14 @@ ra_status launch_backward(const BwdPlan& pl, ra_dtype dt, int S, cudaStream_t st
 }
 
 ra_status launch_delta(const void* o, const void* d_o, ra_dtype dt, int64_t rows, int d, float* delta,
-                       float* zero_rows, cudaStream_t stream) {
+                       cudaStream_t stream) {
   if (rows == 0) return RA_OK;
   int64_t blocks = (rows + DELTA_THREADS / 8 - 1) / (DELTA_THREADS / 8);
   if (blocks > (1ll << 20)) blocks = 1ll << 20;
   if (dt == RA_BF16)
-    bwd_delta_kernel<true><<<(unsigned)blocks, DELTA_THREADS, 0, stream>>>(o, d_o, rows, d, delta, zero_rows);
+    bwd_delta_kernel<true><<<(unsigned)blocks, DELTA_THREADS, 0, stream>>>(o, d_o, rows, d, delta);
   else
-    bwd_delta_kernel<false><<<(unsigned)blocks, DELTA_THREADS, 0, stream>>>(o, d_o, rows, d, delta, zero_rows);
+    bwd_delta_kernel<false><<<(unsigned)blocks, DELTA_THREADS, 0, stream>>>(o, d_o, rows, d, delta);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
@@ -316,7 +322,7 @@ ra_status ra_backward_delta(const void* o, const void* d_o, ra_dtype dt, int64_t
   if (rows == 0) return RA_OK;
   if (!o || !d_o || !delta || !aligned16(o) || !aligned16(d_o) || (reinterpret_cast<uintptr_t>(delta) & 3u))
     return RA_ERR_INVALID_ARG;
-  return launch_delta(o, d_o, dt, rows, d, delta, nullptr, stream);
+  return launch_delta(o, d_o, dt, rows, d, delta, stream);
 }
 
 ra_status ra_partial_backward(const void* q, const void* k, const void* v, const void* d_o, const float* lse,
@@ -341,7 +347,7 @@ ra_status ra_partial_backward(const void* q, const void* k, const void* v, const
   pl.q = q; pl.k = k; pl.v = v; pl.d_o = d_o; pl.lse = lse; pl.delta = delta;
   pl.dq = dq_acc; pl.dk = dk_acc; pl.dv = dv_acc;
   pl.BH = B * H; pl.d = d; pl.P = 1; pl.layout = RA_LAYOUT_CONTIGUOUS; pl.causal = causal;
-  pl.accumulate = 1; pl.dkdv_bf16 = 0;
+  pl.accumulate = 1;
   pl.q_rows = Lq; pl.k_rows = Lk; pl.q_seg_len = Lq; pl.k_seg_len = Lk;
   pl.q_tok0 = q_tok0; pl.q_tok_stride = q_tok_stride; pl.k_tok0 = k_tok0; pl.k_tok_stride = k_tok_stride;
   pl.scale = scale;
@@ -350,9 +356,9 @@ ra_status ra_partial_backward(const void* q, const void* k, const void* v, const
 }
 
 int64_t ra_ring_backward_workspace_bytes(ra_dtype dt, int B, int H, int64_t N, int d) {
+  (void)dt;
   if (B < 0 || H < 0 || N < 0 || d < 1) return -1;
-  const int64_t rows = (int64_t)B * H * N;
-  return dt == RA_BF16 ? rows * (d + 1) * 4 : rows * 4;
+  return (int64_t)B * H * N * 4;  // D, one fp32 per query row
 }
 
 ra_status ra_ring_backward(const void* q, const void* k, const void* v, const void* o, const void* d_o,
@@ -376,27 +382,20 @@ ra_status ra_ring_backward(const void* q, const void* k, const void* v, const vo
       !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(lse) & 3u))
     return RA_ERR_INVALID_ARG;
   const int64_t rows = (int64_t)B * H * N;
-  const bool bf = dt == RA_BF16;
-  float* dq_acc = bf ? static_cast<float*>(workspace) : static_cast<float*>(dq);
-  float* delta = bf ? static_cast<float*>(workspace) + rows * d : static_cast<float*>(workspace);
-  st = launch_delta(o, d_o, dt, rows, d, delta, bf ? dq_acc : nullptr, stream);
+  float* delta = static_cast<float*>(workspace);
+  st = launch_delta(o, d_o, dt, rows, d, delta, stream);
   if (st != RA_OK) return st;
   BwdPlan pl{};
   pl.q = q; pl.k = k; pl.v = v; pl.d_o = d_o; pl.lse = lse; pl.delta = delta;
-  pl.dq = dq_acc; pl.dk = dk; pl.dv = dv;
+  pl.dq = dq; pl.dk = dk; pl.dv = dv;
   pl.BH = B * H; pl.d = d; pl.P = n_chunks; pl.layout = layout; pl.causal = causal;
-  pl.accumulate = 0; pl.dkdv_bf16 = bf ? 1 : 0;
+  pl.accumulate = 0;
   pl.q_rows = N; pl.k_rows = N;
   pl.q_seg_len = pl.k_seg_len = N / parts;
   pl.q_tok0 = 0; pl.q_tok_stride = 1; pl.k_tok0 = 0; pl.k_tok_stride = 1;
   pl.scale = scale;
   pl.scale_log2 = scale * 1.4426950408889634f;
-  st = launch_backward(pl, dt, layout == RA_LAYOUT_STRIPED ? n_chunks : 1, stream);
-  if (st != RA_OK || !bf) return st;
-  int64_t blocks = (rows * d / 4 + 255) / 256;
-  if (blocks > (1ll << 20)) blocks = 1ll << 20;
-  f32_to_bf16_kernel<<<(unsigned)blocks, 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), rows * d / 4);
-  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+  return launch_backward(pl, dt, layout == RA_LAYOUT_STRIPED ? n_chunks : 1, stream);
 }
 
 }  // extern "C"

@@ -139,7 +139,7 @@ def _ring_bwd(lib, **kw):
     (dict(layout=9), binding.RA_ERR_INVALID_ARG),
     (dict(scale=0.0), binding.RA_ERR_INVALID_ARG),
     (dict(d=96), binding.RA_ERR_UNSUPPORTED),
-    (dict(ws_bytes=1000), binding.RA_ERR_INVALID_ARG),               # workspace too small
+    (dict(ws_bytes=1000), binding.RA_ERR_INVALID_ARG),               # workspace too small (needs 2048)
     (dict(ws=None), binding.RA_ERR_INVALID_ARG),
     (dict(lse=ctypes.c_void_p(0x10002)), binding.RA_ERR_INVALID_ARG),
     (dict(dk=ctypes.c_void_p(0x10004)), binding.RA_ERR_INVALID_ARG),
@@ -150,8 +150,8 @@ def test_ring_backward_rejects(lib, kw, code):
 
 def test_ring_backward_workspace_size(lib):
     f = lib.ra_ring_backward_workspace_bytes
-    assert f(1, 1, 2, 256, 128) == 2 * 256 * 129 * 4      # fp32 dQ accumulator + D
-    assert f(0, 1, 2, 256, 16) == 2 * 256 * 4             # D only
+    assert f(1, 1, 2, 256, 128) == 2 * 256 * 4            # D, one fp32 per query row
+    assert f(0, 1, 2, 256, 16) == 2 * 256 * 4
     assert f(1, -1, 2, 256, 128) == -1
     assert _ring_bwd(lib, ws_bytes=f(1, 1, 2, 256, 128) - 1) == binding.RA_ERR_INVALID_ARG
     assert _ring_bwd(lib, N=0) == binding.RA_OK

@@ -44,8 +44,8 @@ def test_noalloc_rejects_problems_beyond_the_scratch():
     """A problem whose workspace exceeds the static array is refused before any launch."""
     lib = binding.load()
     fake = ctypes.c_void_p(0x10000)  # never dereferenced: the size check comes first
-    need = lib.ra_ring_backward_workspace_bytes(binding.RA_BF16, 1, 32, 8192, 128)
+    need = lib.ra_ring_backward_workspace_bytes(binding.RA_BF16, 8, 32, 131072, 128)
     assert need > 64 * 1024 * 1024
-    st = lib.ra_ring_backward_noalloc(fake, fake, fake, fake, fake, fake, binding.RA_BF16, 1, 32, 8192, 128, 0.088,
+    st = lib.ra_ring_backward_noalloc(fake, fake, fake, fake, fake, fake, binding.RA_BF16, 8, 32, 131072, 128, 0.088,
                                       4, 1, 0, fake, fake, fake, None)
     assert st == binding.RA_ERR_UNSUPPORTED
