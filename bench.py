@@ -40,8 +40,10 @@ PROFILE_JSON = os.path.join(ROOT, "profiles", "counters.json")
 KERNEL_SOURCES = {
     "attn_fwd_tc": ["sequence_softmax_b200/csrc/attn_tc.cuh", "sequence_softmax_b200/csrc/common.cuh"],
     "merge": ["sequence_softmax_b200/csrc/merge.cuh"],
-    "attn_bwd_tc": ["sequence_softmax_b200/csrc/bwd_tc.cuh", "sequence_softmax_b200/csrc/bwd.cuh",
-                    "sequence_softmax_b200/csrc/common.cuh"],
+    "attn_bwd_dkdv_tc": ["sequence_softmax_b200/csrc/bwd_tc.cuh", "sequence_softmax_b200/csrc/bwd.cuh",
+                         "sequence_softmax_b200/csrc/common.cuh"],
+    "attn_bwd_dq_tc": ["sequence_softmax_b200/csrc/bwd_dq_tc.cuh", "sequence_softmax_b200/csrc/bwd.cuh",
+                       "sequence_softmax_b200/csrc/common.cuh"],
 }
 BWD_WORKLOAD = "seq128k-d128-causal-zigzag16"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
@@ -410,14 +412,15 @@ def bench_backward(binding, torch, dev, pk, a, rank):
     flops = 2.5 * w.flops()
     tf = flops / (ms / 1e3) / 1e12
     peak = pk["bf16_tflops"]
-    traffic = stored_traffic("attn_bwd_tc", w.name, w.B * w.H * w.N)
+    parts = [stored_traffic(k, w.name, w.B * w.H * w.N) for k in ("attn_bwd_dkdv_tc", "attn_bwd_dq_tc")]
+    traffic = None if any(t is None for t in parts) else sum(parts)
     return {"value": tf, "unit": "TFLOP/s", "ms_per_step": ms, "steps": a.bwd_steps,
             "workload": workload_config(w), "flops_per_step": flops,
             "gpu_launches_per_step": 3,
-            "note": "one step = ra_ring_backward: D + zeroed dQ accumulator, the gradient kernel, dQ to bf16",
+            "note": "one step = ra_ring_backward: D, the dK/dV kernel, the dQ kernel",
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
                          "traffic": traffic, "peak_source": f"{pk['source']} bf16 burst",
-                         "kernel": "attn_bwd_tc_kernel<128> (+ 2 bandwidth-bound launches, ~1% of the step)"},
+                         "kernel": "attn_bwd_dkdv_tc_kernel<128> + attn_bwd_dq_tc_kernel<128> (+ D, <1% of the step)"},
             "wall_s": time.time() - t0}
 
 

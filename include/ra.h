@@ -151,9 +151,9 @@ ra_status ra_backward_delta(const void* o, const void* d_o, ra_dtype dt, int64_t
  *                             softmax probability
  *   delta      [B, H, Lq]     fp32, from ra_backward_delta on the final O
  *   causal and the token arguments as in ra_partial.
- * The bf16 kernel adds dq_acc with atomic vector adds (the order of the additions, and so
- * the last bits of dq_acc, may differ between runs); dk_acc and dv_acc are read, added to
- * and written by the one CTA that owns each key row. Lq == 0 or Lk == 0 is a no-op.
+ * Every row of dq_acc, dk_acc and dv_acc is read, added to and written by the one CTA that
+ * owns it (a key-stationary kernel for dK/dV, a query-stationary one for dQ), so results are
+ * bitwise reproducible. Lq == 0 or Lk == 0 is a no-op.
  */
 ra_status ra_partial_backward(const void* q, const void* k, const void* v, const void* d_o,
                               const float* lse, const float* delta, ra_dtype dt,
@@ -163,16 +163,15 @@ ra_status ra_partial_backward(const void* q, const void* k, const void* v, const
 
 /*
  * ra_ring_backward_workspace_bytes -- bytes of the caller-owned workspace ra_ring_backward
- * needs: B*H*N*(d+1)*4 for bf16 (an fp32 dQ accumulator and D), B*H*N*4 for fp32 (D).
- * Returns -1 for negative sizes.
+ * needs: B*H*N*4 (the row term D, fp32), for either dtype. Returns -1 for negative sizes.
  */
 int64_t ra_ring_backward_workspace_bytes(ra_dtype dt, int B, int H, int64_t N, int d);
 
 /*
  * ra_ring_backward -- gradients of ra_ring_forward's output, by the ring: KV chunk c meets
- * the query positions c, c+1, ... (mod P) in turn; each key tile's dK, dV accumulate on chip
- * and are written once, dQ is accumulated in fp32. Three launches on `stream`: D (and a
- * zeroed dQ accumulator), the gradient kernel(s), and for bf16 the dQ conversion.
+ * the query positions c, c+1, ... (mod P) in turn and each key tile's dK, dV accumulate on
+ * chip; each query tile's dQ accumulates on chip over the KV tiles it sees in the forward's
+ * order. Three launches on `stream`: D, the dK/dV kernel, the dQ kernel. Deterministic.
  *   q, k, v, o, d_o  [B, H, N, d]  dtype dt, natural token order
  *   lse              [B, H, N]     fp32 (from ra_ring_forward)
  *   dq, dk, dv       [B, H, N, d]  dtype dt, written
@@ -193,11 +192,10 @@ ra_status ra_ring_backward(const void* q, const void* k, const void* v, const vo
  * cudaMalloc/cudaFree, which may synchronise the whole device, cannot run. The paper has no
  * counterpart: this is an interface convenience, not part of the method.
  *
- * The scratch (the fp32 dQ accumulator and D) lives in one static device array of
+ * The scratch (the row term D, 4 bytes per query row) lives in one static device array of
  * RA_NOALLOC_SCRATCH_BYTES bytes inside the library. Every GPU that loads the library holds
  * it until the process exits. Problems whose ra_ring_backward_workspace_bytes() exceeds it
- * return RA_ERR_UNSUPPORTED without launching anything (at d = 128 in bf16 the limit is
- * B*H*N <= 130055 rows; fp32 needs only 4 bytes per row).
+ * (B*H*N > 16777216 rows) return RA_ERR_UNSUPPORTED without launching anything.
  *
  * The first call on a device looks up the array's device address, with that device current,
  * and keeps it; make that first call before any stream capture. All calls on a device share

@@ -292,7 +292,7 @@ def ring_backward_noalloc(q, k, v, o, d_o, lse, n_chunks: int, causal: bool = Fa
     """``ring_backward`` through the entry point that allocates nothing on the device.
 
     For callers that cannot allocate device memory: the library's static scratch array
-    replaces the workspace. Pass ``out`` = (dq, dk, dv) preallocated tensors to allocate
+    replaces the workspace (4 bytes per query row, up to 2^24 rows). Pass ``out`` = (dq, dk, dv) preallocated tensors to allocate
     nothing here either. Calls on one device must not overlap on the GPU (they share the
     scratch); problems larger than the array raise RaError(RA_ERR_UNSUPPORTED).
     """

@@ -185,18 +185,12 @@ __device__ __forceinline__ void bwd_exp_row64(uint32_t taddr, const float* nl2co
   }
 }
 
-// ds = bf16 pairs of p_j (dP_j scale + nds_j) = p_j (dP_j - D_j) scale for the 64 fp32 dP
-// columns at taddr; nds_j = -D_j scale is ndscol[j] (per column, shared memory) when PER_COL,
-// else ndsrow. Two paired f32x2 operations per two scores.
+// ds = bf16 pairs of p_j (dP_j scale + nds_j) = p_j (dP_j - D_j) scale for 64 fp32 dP
+// values dr; nds_j = -D_j scale is ndscol[j] (per column, shared memory) when PER_COL, else
+// ndsrow. Two paired f32x2 operations per two scores.
 template <bool PER_COL>
-__device__ __forceinline__ void bwd_ds_row64(uint32_t taddr, const float (&p)[64], const float* ndscol, float ndsrow,
-                                             float scale, uint32_t (&ds)[32]) {
-  uint32_t dr[64];
-  RA_TMEM_LD32(taddr, dr);
-  RA_TMEM_LD32(taddr + 32, (dr + 32));
-  tmem_wait_ld();
-  RA_REG_FENCE32(dr);
-  RA_REG_FENCE32((dr + 32));
+__device__ __forceinline__ void bwd_ds_regs64(const uint32_t (&dr)[64], const float (&p)[64], const float* ndscol,
+                                              float ndsrow, float scale, uint32_t (&ds)[32]) {
   const uint64_t sc2 = f2_pack(scale, scale), z2 = f2_pack(0.f, 0.f);
 #pragma unroll
   for (int j = 0; j < 64; j += 4) {
@@ -211,6 +205,27 @@ __device__ __forceinline__ void bwd_ds_row64(uint32_t taddr, const float (&p)[64
     ds[j / 2] = pack_bf16x2(a, b);
     ds[j / 2 + 1] = pack_bf16x2(c, d);
   }
+}
+
+// As bwd_ds_regs64, with the 64 dP values loaded from the TMEM columns at taddr.
+template <bool PER_COL>
+__device__ __forceinline__ void bwd_ds_row64(uint32_t taddr, const float (&p)[64], const float* ndscol, float ndsrow,
+                                             float scale, uint32_t (&ds)[32]) {
+  uint32_t dr[64];
+  RA_TMEM_LD32(taddr, dr);
+  RA_TMEM_LD32(taddr + 32, (dr + 32));
+  tmem_wait_ld();
+  RA_REG_FENCE32(dr);
+  RA_REG_FENCE32((dr + 32));
+  bwd_ds_regs64<PER_COL>(dr, p, ndscol, ndsrow, scale, ds);
+}
+
+// ceil(num / den) clamped to [0, cap] for num > 0, den >= 1, with a 32-bit division when the
+// result is below the cap (the per-tile causal bound; 64-bit division is slow on the GPU).
+__device__ __forceinline__ int ceil_div_clamped(int64_t num, int64_t den, int cap) {
+  if (num > (int64_t)cap * den) return cap;
+  if (den < (1 << 23)) return (int)(((uint32_t)num + (uint32_t)den - 1u) / (uint32_t)den);
+  return (int)((num + den - 1) / den);
 }
 
 // Epilogue of an fp32 TMEM accumulator row: NC columns at taddr (all lanes of the warp load;

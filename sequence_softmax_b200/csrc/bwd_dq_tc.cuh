@@ -334,9 +334,9 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       // visible key columns of this row: j < hi (tile end, and causally tk0 + tks j <= tq)
       const int64_t tks = pl.k_tok_stride * ks.stride;
       const int64_t tk0 = pl.k_tok0 + pl.k_tok_stride * (ks.row0 + ks.stride * j0);
-      int64_t hi = min((int64_t)BWD_TILE, ks.count - j0);
-      if (pl.causal) hi = tq < tk0 ? 0 : min(hi, (tq - tk0) / tks + 1);
-      const int hl = (int)(hi - c0);  // relative to this thread's first column
+      int hi = (int)min((int64_t)BWD_TILE, ks.count - j0);
+      if (pl.causal) hi = tq < tk0 ? 0 : min(hi, ceil_div_clamped(tq - tk0 + 1, tks, BWD_TILE));
+      const int hl = hi - c0;  // relative to this thread's first column
       const bool masked = !__all_sync(0xffffffffu, hl >= 64);
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full(n & 1), (uint32_t)(n >> 1) & 1u, abort_flag))))
         return false;

@@ -339,10 +339,7 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       const int64_t tq0 = pl.q_tok0 + pl.q_tok_stride * (qs.row0 + qs.stride * i0);
       int lo = 0;
       if (!kvalid) lo = BWD_TILE;
-      else if (pl.causal && tk > tq0) {
-        const int64_t cmin = (tk - tq0 + tqs - 1) / tqs;
-        lo = cmin > BWD_TILE ? BWD_TILE : (int)cmin;
-      }
+      else if (pl.causal && tk > tq0) lo = ceil_div_clamped(tk - tq0, tqs, BWD_TILE);
       // columns c0 .. c0 + 63 of this thread: those below `lo` are masked
       const bool masked = !__all_sync(0xffffffffu, lo <= c0);
       const float* l2s = reinterpret_cast<const float*>(smem + C::LD_OFF + sl * 2 * BWD_TILE * 4) + c0;
