@@ -1,4 +1,5 @@
-"""Ring attention across GPUs: one process per GPU, K and V rotating around the ring.
+"""Ring attention across GPUs: one process per GPU, K and V rotating around the ring
+(forward: ``ring_forward_dist``; backward: ``ring_backward_dist``).
 
 Each rank holds the query, key and value tokens of one virtual ring position (the
 contiguous, striped or zig-zag layout of ``include/ra.h``) and keeps its query block for the
@@ -163,3 +164,73 @@ def ring_forward_dist(q_local, k_local, v_local, N: int, layout: str = "contiguo
         out[:, :, off:off + seg[2]].copy_(parts_o[0])
         lse[:, :, off:off + seg[2]].copy_(parts_l[0])
     return out, lse
+
+
+def _split_segments(t: torch.Tensor, nseg: int):
+    """[B, H, nseg * L, ...] -> list of nseg contiguous [B, H, L, ...] blocks."""
+    L = t.shape[2] // nseg
+    return [t[:, :, s * L:(s + 1) * L].contiguous() for s in range(nseg)]
+
+
+def ring_backward_dist(q_local, k_local, v_local, o_local, do_local, lse_local, N: int, layout: str = "contiguous",
+                       causal: bool = False, scale: float | None = None, group=None, kernels=None):
+    """Gradients (dQ, dK, dV) of ``ring_forward_dist``'s output for upstream gradient do_local.
+
+    Every tensor holds this rank's position tokens as in ``ring_forward_dist``; lse_local is
+    the forward's final lse for them. The ring of "Ring Attention 논문 분석" (youngju.dev),
+    listing ``ring_attention_backward``, with its reduce read as a sum at the owner: each KV
+    block travels with two fp32 accumulators for its dK and dV; at step s the rank holding
+    block (rank - s) mod W adds its queries' contributions to them (``ra_partial_backward``,
+    skipped when the block is wholly in the queries' future) and to its own dQ, then hands
+    the accumulators on. After the last step one more hop brings every block's dK, dV back
+    to its owner. K and V are sent ahead of the step's compute (the transfer overlaps it);
+    the accumulators follow it. ``kernels`` (default: the library binding) provides
+    ``backward_delta`` and ``partial_backward``.
+
+    Returns (dQ, dK, dV) [B, H, N/W, d] in the input dtype.
+    """
+    kern = binding if kernels is None else kernels
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    B, H, n_local, d = q_local.shape
+    segs = position_segments(layout, N, world, rank)
+    nseg = len(segs)
+    if sum(s[2] for s in segs) != n_local or any(t.shape != q_local.shape for t in (k_local, v_local, o_local,
+                                                                                      do_local)):
+        raise ValueError("local tensors must hold the N/W tokens of this rank's position")
+    scale = d ** -0.5 if scale is None else float(scale)
+    dev = q_local.device
+
+    delta = kern.backward_delta(o_local, do_local)
+    q_s, do_s = _split_segments(q_local, nseg), _split_segments(do_local, nseg)
+    lse_s, delta_s = _split_segments(lse_local, nseg), _split_segments(delta, nseg)
+    dq_s = [torch.zeros(q.shape, device=dev, dtype=torch.float32) for q in q_s]
+
+    # Travelling block, segment-major so that every segment is a contiguous [B, H, L, d].
+    kv = torch.stack([torch.stack(_split_segments(k_local, nseg)), torch.stack(_split_segments(v_local, nseg))])
+    acc = torch.zeros(kv.shape, device=dev, dtype=torch.float32)  # dK, dV of the block held
+    kv_next, acc_next = torch.empty_like(kv), torch.empty_like(acc)
+    ex_kv = _Exchanger(group, kv) if world > 1 else None
+    ex_acc = _Exchanger(group, acc) if world > 1 else None
+    for s, src in enumerate(ring_schedule(rank, world)):
+        handle = ex_kv.start(kv, kv_next) if (ex_kv is not None and s < world - 1) else None
+        for ki, kseg in enumerate(position_segments(layout, N, world, src)):
+            for qi, qseg in enumerate(segs):
+                if causal and segment_in_future(qseg, kseg):
+                    continue
+                kern.partial_backward(q_s[qi], kv[0, ki], kv[1, ki], do_s[qi], lse_s[qi], delta_s[qi], dq_s[qi],
+                                      acc[0, ki], acc[1, ki], causal=causal, scale=scale, q_tok0=qseg[0],
+                                      q_tok_stride=qseg[1], k_tok0=kseg[0], k_tok_stride=kseg[1])
+        if ex_acc is not None:
+            # the block's accumulators move on with it; after the last step this hop returns
+            # them to the block's owner
+            acc_next = ex_acc.finish(ex_acc.start(acc, acc_next))
+            acc, acc_next = acc_next, acc
+        if handle is not None:
+            kv_next = ex_kv.finish(handle)
+            kv, kv_next = kv_next, kv
+
+    dq = torch.cat(dq_s, dim=2).to(q_local.dtype)
+    dk = torch.cat(list(acc[0]), dim=2).to(k_local.dtype)
+    dv = torch.cat(list(acc[1]), dim=2).to(v_local.dtype)
+    return dq, dk, dv

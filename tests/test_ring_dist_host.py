@@ -68,3 +68,59 @@ def test_exchange_rotates_blocks(world):
     mp.spawn(_rotate_main, args=(world, port, out), nprocs=world, join=True)
     for r in range(world):
         assert out[r] == ring_dist.ring_schedule(r, world)
+
+
+class _OracleKernels:
+    """Stand-ins for the library's backward kernels on CPU tensors (fp64 oracle), so that the
+    ring's plumbing -- block rotation, accumulator hand-off and the return hop -- runs on gloo
+    ranks without a GPU."""
+
+    @staticmethod
+    def backward_delta(o, d_o):
+        import oracle
+        return torch.from_numpy(oracle.delta(o.numpy(), d_o.numpy())).float()
+
+    @staticmethod
+    def partial_backward(q, k, v, d_o, lse, delta, dq_acc, dk_acc, dv_acc, causal=False, scale=None, q_tok0=0,
+                         q_tok_stride=1, k_tok0=0, k_tok_stride=1):
+        import oracle
+        g = oracle.partial_backward(q.numpy(), k.numpy(), v.numpy(), d_o.numpy(), lse.numpy(), delta.numpy(), scale,
+                                    causal, q_tok0, q_tok_stride, k_tok0, k_tok_stride)
+        for acc, x in zip((dq_acc, dk_acc, dv_acc), g):
+            acc += torch.from_numpy(x).float()
+
+
+def _bwd_main(rank, world, port, layout, causal, out):
+    import oracle
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        B, H, N, d = 1, 2, 24 * world, 8
+        r = np.random.default_rng(5)
+        q, k, v, do = (r.standard_normal((B, H, N, d)).astype(np.float32) for _ in range(4))
+        o, lse = oracle.attention(q, k, v, d ** -0.5, causal)
+        idx = np.concatenate([t0 + st * np.arange(n) for t0, st, n in ring_dist.position_segments(layout, N, world, rank)])
+        loc = lambda x: torch.from_numpy(np.ascontiguousarray(x[:, :, idx])).float()  # noqa: E731
+        g = ring_dist.ring_backward_dist(loc(q), loc(k), loc(v), loc(o), loc(do), loc(lse), N, layout, causal,
+                                         kernels=_OracleKernels)
+        out[rank] = (idx, [t.numpy() for t in g])
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,layout,causal", [(2, "contiguous", True), (3, "zigzag", True), (2, "striped", True),
+                                                 (3, "contiguous", False)])
+def test_ring_backward_plumbing(world, layout, causal):
+    """ring_backward_dist on gloo ranks gives the definition's gradients for every rank's tokens."""
+    import oracle
+    out = mp.get_context("spawn").Manager().dict()
+    port = 29650 + 7 * world + os.getpid() % 400
+    mp.spawn(_bwd_main, args=(world, port, layout, causal, out), nprocs=world, join=True)
+    B, H, N, d = 1, 2, 24 * world, 8
+    r = np.random.default_rng(5)
+    q, k, v, do = (r.standard_normal((B, H, N, d)).astype(np.float32) for _ in range(4))
+    ref = oracle.attention_backward(q, k, v, do, d ** -0.5, causal)
+    for rk in range(world):
+        idx, got = out[rk]
+        for gg, rr in zip(got, ref):
+            assert np.abs(gg - rr[:, :, idx]).max() <= 1e-4 * max(1.0, np.abs(rr).max())
