@@ -106,14 +106,16 @@ class _Exchanger:
 
 
 def ring_forward_dist(q_local, k_local, v_local, N: int, layout: str = "contiguous", causal: bool = False,
-                      scale: float | None = None, group=None):
+                      scale: float | None = None, group=None, kernels=None):
     """Exact attention over a sequence of N tokens split across the ranks of `group`.
 
     q_local, k_local, v_local: [B, H, N/W, d] CUDA tensors (bf16 with d in {64, 128}, or fp32)
     holding the tokens of virtual position `rank` in increasing token order (for zig-zag,
     chunk rank followed by chunk 2W-1-rank). Returns (O_local [B, H, N/W, d] in the input
-    dtype, lse_local [B, H, N/W] fp32) for the same tokens.
+    dtype, lse_local [B, H, N/W] fp32) for the same tokens. ``kernels`` (default: the library
+    binding) provides ``partial`` and ``merge``.
     """
+    kern = binding if kernels is None else kernels
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
     B, H, n_local, d = q_local.shape
@@ -149,9 +151,9 @@ def ring_forward_dist(q_local, k_local, v_local, N: int, layout: str = "contiguo
             for (qs, qseg, _), (parts_o, parts_l) in zip(q_segs, state):
                 if causal and segment_in_future(qseg, kseg):
                     continue
-                binding.partial(qs, kk, vv, causal=causal, scale=scale, q_tok0=qseg[0], q_tok_stride=qseg[1],
-                                k_tok0=kseg[0], k_tok_stride=kseg[1], out=parts_o[1], lse=parts_l[1])
-                merged_o, merged_l = binding.merge(parts_o, parts_l, out_dtype=torch.float32)
+                kern.partial(qs, kk, vv, causal=causal, scale=scale, q_tok0=qseg[0], q_tok_stride=qseg[1],
+                             k_tok0=kseg[0], k_tok_stride=kseg[1], out=parts_o[1], lse=parts_l[1])
+                merged_o, merged_l = kern.merge(parts_o, parts_l, out_dtype=torch.float32)
                 parts_o[0].copy_(merged_o)
                 parts_l[0].copy_(merged_l)
         if handle is not None:
