@@ -332,7 +332,7 @@ def main():
     torch.cuda.empty_cache()
 
     if not a.no_backward:
-        line["backward"] = bench_backward(binding, torch, dev, pk, a, rank)
+        line["backward"] = bench_backward(binding, torch, dev, pk, a, rank, world)
         torch.cuda.empty_cache()
 
     if rank == 0 and not a.no_cpu_baseline and world == 1:
@@ -376,9 +376,11 @@ def bench_merge(binding, torch, dev, pk, a):
                          "peak_source": f"{pk['source']} copy"}}
 
 
-def bench_backward(binding, torch, dev, pk, a, rank):
+def bench_backward(binding, torch, dev, pk, a, rank, world=1):
     """ra_ring_backward on its own workload: dQ, dK, dV of the forward's output for a seeded
-    upstream gradient. FLOPs = 2.5x the forward's (five GEMMs per visible pair instead of two)."""
+    upstream gradient. FLOPs = 2.5x the forward's (five GEMMs per visible pair instead of two).
+    With N ranks each runs its own replica; the step time is the slowest rank's and the value
+    is the whole job's throughput (weak scaling, as the headline)."""
     from sequence_softmax_b200.inputs import WORKLOADS, make_qkv, workload_qkv
     w = WORKLOADS[a.bwd_workload]
     q, k, v = workload_qkv(w, device=dev, batch_offset=rank)
@@ -408,9 +410,10 @@ def bench_backward(binding, torch, dev, pk, a, rank):
         kernel_ms.append(s.elapsed_time(e))
     if binding.get_device_error() != binding.RA_OK:
         raise RuntimeError("device error in the timed backward")
-    ms = statistics.median(kernel_ms)
+    ms = max_over_ranks(statistics.median(kernel_ms), world, dev)
     flops = 2.5 * w.flops()
-    tf = flops / (ms / 1e3) / 1e12
+    tf = world * flops / (ms / 1e3) / 1e12
+    per_gpu = flops / (ms / 1e3) / 1e12
     peak = pk["bf16_tflops"]
     parts = [stored_traffic(k, w.name, w.B * w.H * w.N) for k in ("attn_bwd_dkdv_tc", "attn_bwd_dq_tc")]
     traffic = None if any(t is None for t in parts) else sum(parts)
@@ -418,7 +421,8 @@ def bench_backward(binding, torch, dev, pk, a, rank):
             "workload": workload_config(w), "flops_per_step": flops,
             "gpu_launches_per_step": 3,
             "note": "one step = ra_ring_backward: D, the dK/dV kernel, the dQ kernel",
-            "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+            "roofline": {"bound": "tensor", "achieved": per_gpu, "peak": peak, "unit": "TFLOP/s",
+                         "frac": per_gpu / peak,
                          "traffic": traffic, "peak_source": f"{pk['source']} bf16 burst",
                          "kernel": "attn_bwd_dkdv_tc_kernel<128> + attn_bwd_dq_tc_kernel<128> (+ D, <1% of the step)"},
             "wall_s": time.time() - t0}
