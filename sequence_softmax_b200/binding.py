@@ -161,28 +161,75 @@ def merge(o_parts, lse_parts, out_dtype=torch.bfloat16, with_lse: bool = True, o
     return out, (lse if with_lse else None)
 
 
+HOST_PIPELINE_GROUPS = 4
+
+
+def _ring_forward_host(q, k, v, n_chunks, causal, layout, scale, return_lse, out, lse, stream):
+    """ring_forward for host tensors: the (batch, head) rows are processed in up to
+    HOST_PIPELINE_GROUPS groups, one library call each, so that the copy of group g + 1's
+    inputs to the device and of group g - 1's outputs back to the host (on two copy streams)
+    overlap group g's kernel. Heads are independent, so the result equals one call over all
+    heads. With pinned host tensors the copies are asynchronous; otherwise they serialise."""
+    for t, n in ((k, "k"), (v, "v")):
+        if t.is_cuda or t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError(f"{n} must be a host tensor shaped and typed like q")
+    if not all(t.is_contiguous() for t in (q, k, v)):
+        raise ValueError("host q, k, v must be contiguous")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    B, H, N, d = q.shape
+    BH = B * H
+    pin = q.is_pinned() and k.is_pinned() and v.is_pinned()
+    o_h = torch.empty(q.shape, dtype=q.dtype, pin_memory=pin) if out is None else out
+    l_h = None
+    if return_lse:
+        l_h = torch.empty(B, H, N, dtype=torch.float32, pin_memory=pin) if lse is None else lse
+    if BH == 0 or N == 0:
+        return o_h, l_h
+    qf, kf, vf, of = (t.view(BH, N, d) for t in (q, k, v, o_h))
+    lf = l_h.view(BH, N) if return_lse else None
+    qd, kd, vd, od = (torch.empty(BH, N, d, dtype=q.dtype, device=dev) for _ in range(4))
+    ld = torch.empty(BH, N, dtype=torch.float32, device=dev) if return_lse else None
+    compute = torch.cuda.current_stream() if stream is None else stream
+    h2d, d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    G = max(1, min(HOST_PIPELINE_GROUPS, BH))
+    bounds = [BH * g // G for g in range(G + 1)]
+    for g in range(G):
+        a, b = bounds[g], bounds[g + 1]
+        if a == b:
+            continue
+        with torch.cuda.stream(h2d):
+            for dst, src in ((qd, qf), (kd, kf), (vd, vf)):
+                dst[a:b].copy_(src[a:b], non_blocking=pin)
+            loaded = torch.cuda.Event()
+            loaded.record(h2d)
+        compute.wait_event(loaded)
+        view = lambda t: t[a:b].view(1, b - a, N, d)  # noqa: E731
+        ring_forward(view(qd), view(kd), view(vd), n_chunks, causal, layout, scale, return_lse, out=view(od),
+                     lse=ld[a:b].view(1, b - a, N) if return_lse else None, stream=compute)
+        done = torch.cuda.Event()
+        done.record(compute)
+        d2h.wait_event(done)
+        with torch.cuda.stream(d2h):
+            of[a:b].copy_(od[a:b], non_blocking=pin)
+            if return_lse:
+                lf[a:b].copy_(ld[a:b], non_blocking=pin)
+    d2h.synchronize()
+    compute.synchronize()
+    return o_h, l_h
+
+
 def ring_forward(q, k, v, n_chunks: int, causal: bool = False, layout: str = "contiguous",
                  scale: float | None = None, return_lse: bool = True, out=None, lse=None, stream=None):
     """Exact attention by the ordered ring over ``n_chunks`` virtual positions.
 
     q, k, v [B, H, N, d] (bf16 with d in {64, 128}, or fp32 with d <= 128), natural token order.
     Returns (O [B,H,N,d] in q's dtype, lse [B,H,N] fp32 or None). Host (CPU) tensors are
-    accepted: they are copied to the current device, the call runs there, and the results
-    are copied back to host memory before returning.
+    accepted: they are copied to the current device group of heads by group, overlapped with
+    the computation of the previous group, and the results are copied back to host memory
+    before returning.
     """
     if not q.is_cuda:
-        dev = torch.device("cuda", torch.cuda.current_device())
-        qd, kd, vd = (t.to(dev, non_blocking=True) for t in (q, k, v))
-        o_d, l_d = ring_forward(qd, kd, vd, n_chunks, causal, layout, scale, return_lse, stream=stream)
-        pin = q.is_pinned()
-        o_h = torch.empty(o_d.shape, dtype=o_d.dtype, pin_memory=pin) if out is None else out
-        o_h.copy_(o_d, non_blocking=pin)
-        l_h = None
-        if return_lse:
-            l_h = torch.empty(l_d.shape, dtype=l_d.dtype, pin_memory=pin) if lse is None else lse
-            l_h.copy_(l_d, non_blocking=pin)
-        torch.cuda.current_stream().synchronize()
-        return o_h, l_h
+        return _ring_forward_host(q, k, v, n_chunks, causal, layout, scale, return_lse, out, lse, stream)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _dev(t, n)
     B, H, N, d = q.shape

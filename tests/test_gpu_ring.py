@@ -89,6 +89,18 @@ def test_host_buffers_round_trip(cuda):
     compare(to_np(o), to_np(lse), o_ref, lse_ref, "bf16", "host buffers")
 
 
+@pytest.mark.parametrize("pinned", [True, False])
+def test_host_pipeline_equals_device_call(cuda, pinned):
+    """The host path runs the (batch, head) rows in groups with copies overlapped; heads are
+    independent, so it must equal one device call bit for bit (6 rows in 4 uneven groups)."""
+    q, k, v = make_qkv(2, 3, 1024, 128, torch.bfloat16, seed=18, device="cpu")
+    if pinned:
+        q, k, v = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    o_h, l_h = binding.ring_forward(q, k, v, 4, True, "zigzag")
+    o_d, l_d = binding.ring_forward(q.cuda(), k.cuda(), v.cuda(), 4, True, "zigzag")
+    assert torch.equal(o_h, o_d.cpu()) and torch.equal(l_h, l_d.cpu())
+
+
 @pytest.mark.parametrize("name", ["seq4k-d64-noncausal-8chunks", "seq4k-d64-noncausal-8chunks-qx4"])
 def test_workload_full_compare(cuda, name):
     w = WORKLOADS[name]
