@@ -41,6 +41,7 @@ attn_fwd_simt_f32_kernel(const Plan pl, int64_t rows_per_pos) {
   const int si = (int)(li / pl.q_seg_len);
   const Seg qs = segment_of(pl.layout, pl.P, pl.q_seg_len, p, si);
   const int64_t qrow = qs.row0 + qs.stride * (li - (int64_t)si * pl.q_seg_len);
+  if (!in_bounds(qrow < pl.q_rows && bh < pl.BH)) return;  // whole warp: qrow is warp-uniform
   const int64_t tq = pl.q_tok0 + pl.q_tok_stride * qrow;
   const float* qp = static_cast<const float*>(pl.q) + ((int64_t)bh * pl.q_rows + qrow) * d;
   const float* kb = static_cast<const float*>(pl.k) + (int64_t)bh * pl.k_rows * d;
@@ -63,7 +64,8 @@ attn_fwd_simt_f32_kernel(const Plan pl, int64_t rows_per_pos) {
       for (int64_t j0 = 0; j0 < nvis; j0 += 32) {
         const int64_t j = j0 + lane;
         const int64_t krow = ks.row0 + ks.stride * j;
-        const bool vis = j < nvis && (!pl.causal || pl.k_tok0 + pl.k_tok_stride * krow <= tq);
+        const bool vis = j < nvis && in_bounds(krow < pl.k_rows) &&
+                         (!pl.causal || pl.k_tok0 + pl.k_tok_stride * krow <= tq);
         float sc = -INFINITY;
         if (vis) {
           const float* kp = kb + krow * d;

@@ -261,6 +261,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (lane == 0) {
       const int qy = (int)(qb.seg.row0 % qb.seg.stride);
       const int64_t qz0 = qb.seg.row0 / qb.seg.stride + qb.i0;
+      // the block starts inside its segment and the segment lies inside the tensor
+      in_bounds(qb.i0 < qb.seg.count && qb.seg.row0 + qb.seg.stride * (qb.seg.count - 1) < pl.q_rows &&
+                bh < pl.BH);
       for (int t = 0; t < 2; ++t) {
         mbar_arrive_expect_tx(bar_q_full(t), C::TILE_BYTES);
         for (int b = 0; b < C::NBOX; ++b)
@@ -278,6 +281,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           const int ky = (int)(ks.row0 % ks.stride);
           const int64_t kz0 = ks.row0 / ks.stride;
           for (int jt = 0; jt < ntiles && ok; ++jt) {
+            in_bounds((int64_t)jt * TC_BN < ks.count && ks.row0 + ks.stride * (ks.count - 1) < pl.k_rows);
             for (int kv = 0; kv < 2; ++kv, ++use) {
               const int st = use % C::NSTAGE;
               const uint32_t ph = (use / C::NSTAGE) & 1u;
@@ -512,6 +516,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const int64_t mrow = qb.seg.row0 + qb.seg.stride * li;
       const int64_t orow = (int64_t)bh * pl.q_rows + mrow;
+      const bool row_ok = row_valid && in_bounds(mrow < pl.q_rows);
       if (T > 0) tc_fence_after_sync();
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
@@ -524,7 +529,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
           for (int j = 0; j < 32; ++j) orr[j] = 0u;
         }
-        if (row_valid) {
+        if (row_ok) {
           if (pl.out_f32) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(pl.o) + orow * D + cc * 32);
 #pragma unroll
@@ -545,7 +550,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           }
         }
       }
-      if (row_valid && pl.lse != nullptr)
+      if (row_ok && pl.lse != nullptr)
         pl.lse[orow] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
     }
   }

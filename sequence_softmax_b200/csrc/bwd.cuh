@@ -296,6 +296,7 @@ bwd_dkdv_simt_f32_kernel(const BwdPlan pl, int64_t rows_per_pos) {
   const int sk_i = (int)(lj / pl.k_seg_len);
   const Seg ks = segment_of(pl.layout, pl.P, pl.k_seg_len, c, sk_i);
   const int64_t krow = ks.row0 + ks.stride * (lj - (int64_t)sk_i * pl.k_seg_len);
+  if (!in_bounds(krow < pl.k_rows && bh < pl.BH)) return;  // whole warp: krow is warp-uniform
   const int64_t tk = pl.k_tok0 + pl.k_tok_stride * krow;
   const float* kp = static_cast<const float*>(pl.k) + ((int64_t)bh * pl.k_rows + krow) * d;
   const float* vp = static_cast<const float*>(pl.v) + ((int64_t)bh * pl.k_rows + krow) * d;
@@ -322,7 +323,7 @@ bwd_dkdv_simt_f32_kernel(const BwdPlan pl, int64_t rows_per_pos) {
         const int64_t i = i0 + lane;
         const int64_t qrow = qs.row0 + qs.stride * i;
         float pij = 0.f, dsij = 0.f;
-        if (i < qs.count && (!pl.causal || tk <= pl.q_tok0 + pl.q_tok_stride * qrow)) {
+        if (i < qs.count && in_bounds(qrow < pl.q_rows) && (!pl.causal || tk <= pl.q_tok0 + pl.q_tok_stride * qrow)) {
           const float* qp = qb + qrow * d;
           const float* op = ob + qrow * d;
           float dot = 0.f, dpd = 0.f;
@@ -385,6 +386,7 @@ bwd_dq_simt_f32_kernel(const BwdPlan pl, int64_t rows_per_pos) {
   const int si = (int)(li / pl.q_seg_len);
   const Seg qs = segment_of(pl.layout, pl.P, pl.q_seg_len, p, si);
   const int64_t qrow = qs.row0 + qs.stride * (li - (int64_t)si * pl.q_seg_len);
+  if (!in_bounds(qrow < pl.q_rows && bh < pl.BH)) return;  // whole warp: qrow is warp-uniform
   const int64_t tq = pl.q_tok0 + pl.q_tok_stride * qrow;
   const float* qp = static_cast<const float*>(pl.q) + ((int64_t)bh * pl.q_rows + qrow) * d;
   const float* op = static_cast<const float*>(pl.d_o) + ((int64_t)bh * pl.q_rows + qrow) * d;
@@ -417,7 +419,7 @@ bwd_dq_simt_f32_kernel(const BwdPlan pl, int64_t rows_per_pos) {
         const int64_t j = j0 + lane;
         const int64_t krow = ks.row0 + ks.stride * j;
         float dsij = 0.f;
-        if (j < nvis && (!pl.causal || pl.k_tok0 + pl.k_tok_stride * krow <= tq)) {
+        if (j < nvis && in_bounds(krow < pl.k_rows) && (!pl.causal || pl.k_tok0 + pl.k_tok_stride * krow <= tq)) {
           const float* kr = kb + krow * d;
           const float* vr = vb + krow * d;
           float dot = 0.f, dpd = 0.f;

@@ -199,6 +199,8 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   if (warp == BQ_WARP_PRODUCER) {
     // ------------------------------------------------------------------ producer
     if (T > 0 && lane == 0) {
+      in_bounds(qt.i0 < qt.seg.count && qt.seg.row0 + qt.seg.stride * (qt.seg.count - 1) < pl.q_rows &&
+                bh < pl.BH);
       mbar_arrive_expect_tx(bar_qo_full, 2 * C::TILE_BYTES);
       const int qy = (int)(qt.seg.row0 % qt.seg.stride);
       const int qz = (int)(qt.seg.row0 / qt.seg.stride + qt.i0);
@@ -211,6 +213,7 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const int n = issued, sk = n % C::NK, sv = n % C::NV;
         const int ky = (int)(ks.row0 % ks.stride);
         const int kz = (int)(ks.row0 / ks.stride + j0);
+        in_bounds(j0 < ks.count && ks.row0 + ks.stride * (ks.count - 1) < pl.k_rows);
         if (!mbar_wait(bar_k_empty(sk), ((uint32_t)(n / C::NK) & 1u) ^ 1u, abort_flag)) return false;
         mbar_arrive_expect_tx(bar_k_full(sk), C::TILE_BYTES);
         for (int b = 0; b < C::NBOX; ++b)
@@ -317,8 +320,8 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const int c0 = 64 * g;  // this thread's key columns of S / dP
     const int64_t li = qt.i0 + row;
-    const bool qvalid = li < qt.seg.count;
     const int64_t qrow = qt.seg.row0 + qt.seg.stride * li;
+    const bool qvalid = li < qt.seg.count && in_bounds(qrow < pl.q_rows);
     const int64_t tq = pl.q_tok0 + pl.q_tok_stride * qrow;
     float nl2row = -INFINITY, ndsrow = 0.f;  // rows past the segment end (or that saw no key): P = 0
     if (qvalid) {

@@ -161,6 +161,8 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     // ------------------------------------------------------------------ producer
     if (T > 0) {
       if (lane == 0) {
+        in_bounds(kt.j0 < kt.seg.count && kt.seg.row0 + kt.seg.stride * (kt.seg.count - 1) < pl.k_rows &&
+                  bh < pl.BH);
         mbar_arrive_expect_tx(bar_kv_full, 2 * C::TILE_BYTES);
         const int ky = (int)(kt.seg.row0 % kt.seg.stride);
         const int kz = (int)(kt.seg.row0 / kt.seg.stride + kt.j0);
@@ -183,8 +185,9 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           const bool v = li < qs.count;
           ld_valid |= (v ? 1u : 0u) << m;
           const int64_t idx = (int64_t)bh * pl.q_rows + qs.row0 + qs.stride * (v ? li : 0);
-          ld_l[m] = pl.lse[idx];
-          ld_d[m] = pl.delta[idx];
+          const bool ok = in_bounds(qs.row0 + qs.stride * (v ? li : 0) < pl.q_rows);
+          ld_l[m] = ok ? pl.lse[idx] : -INFINITY;
+          ld_d[m] = ok ? pl.delta[idx] : 0.f;
         }
       };
       auto store_ld = [&](int u) {  // tile u's values into slot u & 1
@@ -212,6 +215,7 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         const int qy = (int)(qs.row0 % qs.stride);
         const int qz = (int)(qs.row0 / qs.stride + i0);
         if (lane == 0) {
+          in_bounds(i0 < qs.count && qs.row0 + qs.stride * (qs.count - 1) < pl.q_rows);
           mbar_arrive_expect_tx(bar_q_full(sq), C::TILE_BYTES);
           for (int b = 0; b < C::NBOX; ++b)
             tma_load_4d(sQ(sq) + b * C::BOX_BYTES, &tm_q, bar_q_full(sq), 64 * b, qy, qz, bh);
@@ -379,9 +383,10 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       if (T > 0) tc_fence_after_sync();
       const int64_t krow = kt.seg.row0 + kt.seg.stride * jl;
       const int64_t off = ((int64_t)bh * pl.k_rows + krow) * D + g * (D / 2);
-      bwd_store_acc_row<D / 2>(tmem + C::COL_DV + lane_off + g * (D / 2), T > 0, kvalid, pl.dv, off,
+      const bool row_ok = kvalid && in_bounds(krow < pl.k_rows);
+      bwd_store_acc_row<D / 2>(tmem + C::COL_DV + lane_off + g * (D / 2), T > 0, row_ok, pl.dv, off,
                                pl.accumulate != 0);
-      bwd_store_acc_row<D / 2>(tmem + C::COL_DK + lane_off + g * (D / 2), T > 0, kvalid, pl.dk, off,
+      bwd_store_acc_row<D / 2>(tmem + C::COL_DK + lane_off + g * (D / 2), T > 0, row_ok, pl.dk, off,
                                pl.accumulate != 0);
     }
   }

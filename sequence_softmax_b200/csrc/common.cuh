@@ -22,6 +22,21 @@ __device__ unsigned g_error_word = 0;
 
 __device__ __forceinline__ void record_error(unsigned bits) { atomicOr(&g_error_word, bits); }
 
+// Checked builds (compiled with -DRA_DEBUG_BOUNDS, as libra_checked.so): the kernels test
+// every global row index and every TMA start row they compute against the buffer it
+// addresses. A failed test records DEVERR_BOUNDS in the error word (RA_ERR_DEVICE_BOUNDS on
+// the host) and the access is skipped; TMA loads, whose out-of-range parts read as zeros,
+// are still issued so that no wait is left without its data. The default build compiles
+// the tests away.
+#ifdef RA_DEBUG_BOUNDS
+__device__ __forceinline__ bool in_bounds(bool ok) {
+  if (!ok) record_error(DEVERR_BOUNDS);
+  return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool in_bounds(bool) { return true; }
+#endif
+
 // Time limit of every spin on an mbarrier (nanoseconds of %globaltimer). A correct kernel
 // waits microseconds; the limit turns a lost arrival into an error instead of a hang.
 #ifndef RA_WAIT_LIMIT_NS

@@ -4,6 +4,8 @@
 #include <mutex>
 #include <stdio.h>
 
+#include <nvtx3/nvToolsExt.h>  // header-only; a profiler that is attached sees one range per call
+
 #include "common.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
@@ -31,6 +33,15 @@ __global__ void selftest_wait_timeout_kernel(uint64_t limit_ns) {
 }
 
 namespace {
+
+// An NVTX range over one entry point (named after it) for timeline tools; without a tool
+// attached the push and pop are no-ops.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // ---- cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda) ----
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -224,6 +235,7 @@ ra_status ra_get_device_error(cudaStream_t stream) {
 }
 
 ra_status ra_selftest_wait_timeout(int64_t limit_ns, cudaStream_t stream) {
+  NvtxRange nvtx_range("ra_selftest_wait_timeout");
   if (limit_ns < 1000000 || limit_ns > 2000000000) return RA_ERR_INVALID_ARG;
   selftest_wait_timeout_kernel<<<1, 32, 0, stream>>>((uint64_t)limit_ns);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
@@ -232,6 +244,7 @@ ra_status ra_selftest_wait_timeout(int64_t limit_ns, cudaStream_t stream) {
 ra_status ra_partial(const void* q, const void* k, const void* v, ra_dtype dt, int B, int H, int64_t Lq,
                      int64_t Lk, int d, float scale, int causal, int64_t q_tok0, int64_t q_tok_stride,
                      int64_t k_tok0, int64_t k_tok_stride, float* o_partial, float* lse, cudaStream_t stream) {
+  NvtxRange nvtx_range("ra_partial");
   if (B < 0 || H < 0 || Lq < 0 || Lk < 0) return RA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return RA_ERR_INVALID_ARG;
@@ -259,6 +272,7 @@ ra_status ra_partial(const void* q, const void* k, const void* v, ra_dtype dt, i
 
 ra_status ra_merge(const float* o_parts, const float* lse_parts, int n, int64_t rows, int d, void* o_out,
                    ra_dtype out_dt, float* lse_out, cudaStream_t stream) {
+  NvtxRange nvtx_range("ra_merge");
   if (n < 1 || rows < 0 || d < 1 || (d & 3) != 0) return RA_ERR_INVALID_ARG;
   if (out_dt != RA_F32 && out_dt != RA_BF16) return RA_ERR_INVALID_ARG;
   if (n > MERGE_MAX_PARTS) return RA_ERR_UNSUPPORTED;
@@ -288,6 +302,7 @@ ra_status ra_merge(const float* o_parts, const float* lse_parts, int n, int64_t 
 ra_status ra_ring_forward(const void* q, const void* k, const void* v, ra_dtype dt, int B, int H, int64_t N, int d,
                           float scale, int n_chunks, int causal, ra_layout layout, void* o, float* lse,
                           cudaStream_t stream) {
+  NvtxRange nvtx_range("ra_ring_forward");
   if (B < 0 || H < 0 || N < 0 || n_chunks < 1) return RA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return RA_ERR_INVALID_ARG;
@@ -316,6 +331,7 @@ ra_status ra_ring_forward(const void* q, const void* k, const void* v, ra_dtype 
 
 ra_status ra_backward_delta(const void* o, const void* d_o, ra_dtype dt, int64_t rows, int d, float* delta,
                             cudaStream_t stream) {
+  NvtxRange nvtx_range("ra_backward_delta");
   if (rows < 0) return RA_ERR_INVALID_ARG;
   ra_status st = check_dtype_d(dt, d);
   if (st != RA_OK) return st;
@@ -330,6 +346,7 @@ ra_status ra_partial_backward(const void* q, const void* k, const void* v, const
                               float scale, int causal, int64_t q_tok0, int64_t q_tok_stride, int64_t k_tok0,
                               int64_t k_tok_stride, float* dq_acc, float* dk_acc, float* dv_acc,
                               cudaStream_t stream) {
+  NvtxRange nvtx_range("ra_partial_backward");
   if (B < 0 || H < 0 || Lq < 0 || Lk < 0) return RA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return RA_ERR_INVALID_ARG;
@@ -365,6 +382,7 @@ ra_status ra_ring_backward(const void* q, const void* k, const void* v, const vo
                            const float* lse, ra_dtype dt, int B, int H, int64_t N, int d, float scale,
                            int n_chunks, int causal, ra_layout layout, void* dq, void* dk, void* dv,
                            void* workspace, int64_t workspace_bytes, cudaStream_t stream) {
+  NvtxRange nvtx_range("ra_ring_backward");
   if (B < 0 || H < 0 || N < 0 || n_chunks < 1) return RA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return RA_ERR_INVALID_ARG;
@@ -433,6 +451,7 @@ extern "C" ra_status ra_ring_backward_noalloc(const void* q, const void* k, cons
                                               int64_t N, int d, float scale, int n_chunks, int causal,
                                               ra_layout layout, void* dq, void* dk, void* dv,
                                               cudaStream_t stream) {
+  NvtxRange nvtx_range("ra_ring_backward_noalloc");
   const int64_t need = ra_ring_backward_workspace_bytes(dt, B, H, N, d);
   if (need < 0) return RA_ERR_INVALID_ARG;
   if (need > RA_NOALLOC_SCRATCH_BYTES) return RA_ERR_UNSUPPORTED;

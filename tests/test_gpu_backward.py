@@ -141,3 +141,15 @@ def test_backward_delta(cuda, kind, d):
     got = to_np(binding.backward_delta(o, do))
     ref = oracle.delta(to_np(o), to_np(do))
     assert np.abs(got - ref).max() <= 1e-5 * (1 + np.abs(ref).max())
+
+
+def test_ring_backward_is_deterministic(cuda):
+    """Every row of dQ, dK and dV is produced by exactly one CTA (no reductions into shared
+    memory between CTAs), so two runs agree bit for bit."""
+    q, k, v = make_qkv(1, 4, 2048, 128, torch.bfloat16, seed=41, device="cuda")
+    do = _upstream(1, 4, 2048, 128, torch.bfloat16, seed=42)
+    o, lse = binding.ring_forward(q, k, v, 4, True, "zigzag")
+    a = binding.ring_backward(q, k, v, o, do, lse, 4, True, "zigzag")
+    b = binding.ring_backward(q, k, v, o, do, lse, 4, True, "zigzag")
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
