@@ -14,6 +14,12 @@ Recipe:
   [B, H, N, d], i.i.d. N(0, 1), then cast to the workload dtype. A query scale (the
   "Q x 4" running-max stress case) is applied after the cast; scaling by a power of two
   is exact in bf16.
+* Score ramp (``ramp_qkv``): every query is 4u plus small noise and every key of 128-key
+  block b is (b x gamma) u plus a random component orthogonal to u (8 N(0, 1) per
+  coordinate, projected), for one random unit vector u; V is N(0, 1).
+  A query's largest score then grows by about ``jump_log2`` (in log2 units, at the default
+  scale d^-1/2) from each key block to the next, so an online softmax that visits the
+  blocks in token order sees its running maximum move at every block.
 """
 
 from __future__ import annotations
@@ -119,3 +125,30 @@ def sample_rows(N: int, n_chunks: int, layout: str, count: int = 4096, seed: int
         edges += [i * c - 1, i * c]
     rows = torch.unique(torch.cat([rnd, torch.tensor(edges)]))
     return rows.numpy()
+
+
+RAMP_BLOCK = 128  # keys per block of the score ramp
+
+
+def ramp_qkv(N: int, d: int, jump_log2: float, seed: int = 0, dtype=torch.bfloat16, device="cpu",
+             B: int = 1, H: int = 1):
+    """Seeded q, k, v [B, H, N, d] whose scores rise by ~jump_log2 per 128-key block.
+
+    q_i = 4 u + 0.02 n_i, k_j = (floor(j / 128) gamma) u + 8 (I - u u^T) n'_j with gamma
+    chosen so that 4 gamma d^-1/2 log2(e) = jump_log2; u is a unit vector, n, n' i.i.d.
+    N(0, 1). The orthogonal part barely moves the scores (the queries are nearly parallel to
+    u) but keeps the keys of one block apart: without it every key of the dominant block is
+    the same vector, the rows of dS (which sum to zero) multiply it, and dQ is a small
+    difference of large terms.
+    """
+    g = torch.Generator().manual_seed(seed)
+    u = torch.randn(d, generator=g, dtype=torch.float64)
+    u /= u.norm()
+    a = 4.0
+    gamma = jump_log2 / (a * d ** -0.5 * 1.4426950408889634)
+    block = (torch.arange(N, dtype=torch.float64) // RAMP_BLOCK)[:, None]
+    q = a * u + 0.02 * torch.randn(B, H, N, d, generator=g, dtype=torch.float64)
+    w = torch.randn(B, H, N, d, generator=g, dtype=torch.float64)
+    k = gamma * block * u + 8.0 * (w - (w @ u)[..., None] * u)
+    v = torch.randn(B, H, N, d, generator=g, dtype=torch.float64)
+    return tuple(t.to(dtype).to(device) for t in (q, k, v))

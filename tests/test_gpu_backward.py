@@ -11,7 +11,7 @@ import torch
 
 import oracle
 from sequence_softmax_b200 import binding
-from sequence_softmax_b200.inputs import make_qkv
+from sequence_softmax_b200.inputs import make_qkv, ramp_qkv
 
 from .parity import compare_grads, to_np
 
@@ -49,6 +49,21 @@ def test_ring_backward_matches_oracle(cuda, case):
     assert binding.get_device_error() == binding.RA_OK
     ref = oracle.attention_backward(to_np(q), to_np(k), to_np(v), to_np(do), d ** -0.5, causal)
     print(case, compare_grads((to_np(dq), to_np(dk), to_np(dv)), ref, kind, str(case)))
+
+
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag"])
+def test_ring_backward_on_rising_scores(cuda, layout):
+    """The score ramp (every 128-key block scores ~10 log2 units above the one before): the
+    forward rescales its running state at every block and the backward rebuilds P from the
+    final lse."""
+    N, d, P = 1024, 128, 4
+    q, k, v = ramp_qkv(N, d, 10.0, seed=7, device="cuda")
+    do = _upstream(1, 1, N, d, torch.bfloat16, seed=8)
+    o, lse = binding.ring_forward(q, k, v, P, True, layout)
+    dq, dk, dv = binding.ring_backward(q, k, v, o, do, lse, P, True, layout)
+    assert binding.get_device_error() == binding.RA_OK
+    ref = oracle.attention_backward(to_np(q), to_np(k), to_np(v), to_np(do), d ** -0.5, True)
+    print(layout, compare_grads((to_np(dq), to_np(dk), to_np(dv)), ref, "bf16", layout))
 
 
 def test_ring_backward_layout_invariant(cuda):

@@ -12,7 +12,7 @@ import torch
 
 import oracle
 from sequence_softmax_b200 import binding
-from sequence_softmax_b200.inputs import WORKLOADS, make_qkv, sample_rows, workload_qkv
+from sequence_softmax_b200.inputs import WORKLOADS, make_qkv, ramp_qkv, sample_rows, workload_qkv
 
 from .parity import compare, to_np
 
@@ -60,6 +60,30 @@ def test_ring_matches_oracle(cuda, case):
     assert binding.get_device_error() == binding.RA_OK
     o_ref, lse_ref = oracle.attention(to_np(q), to_np(k), to_np(v), d ** -0.5, causal)
     compare(to_np(o), to_np(lse), o_ref, lse_ref, kind, str(case))
+
+
+RAMP_CASES = [
+    # jump (log2 units per 128-key block), N, d, P, layout, causal
+    (10.0, 1024, 128, 1, "contiguous", False),  # the running max moves past the threshold every block
+    (6.0, 1024, 128, 1, "contiguous", True),    # moves by less than the threshold, then past it
+    (10.0, 1024, 64, 1, "contiguous", True),
+    (10.0, 2048, 128, 4, "contiguous", False),  # ring order: a big jump when the walk wraps
+    (10.0, 2048, 128, 4, "zigzag", True),
+    (6.0, 2048, 128, 4, "striped", True),
+]
+
+
+@pytest.mark.parametrize("case", RAMP_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_running_max_rescale_matches_oracle(cuda, case):
+    """Scores that rise block after block (the score ramp of the inputs module) make the
+    forward move its running maximum, and rescale O and l, while it walks the keys."""
+    jump, N, d, P, layout, causal = case
+    q, k, v = ramp_qkv(N, d, jump, seed=N + P, device="cuda")
+    o, lse = binding.ring_forward(q, k, v, P, causal, layout)
+    assert binding.get_device_error() == binding.RA_OK
+    o_ref, lse_ref = oracle.attention(to_np(q), to_np(k), to_np(v), d ** -0.5, causal)
+    assert np.abs(o_ref).mean() > 10 * 2e-3  # a wrong rescale moves O by far more than the mean tolerance
+    compare(to_np(o), to_np(lse), o_ref, lse_ref, "bf16", str(case))
 
 
 def test_layout_invariance_on_gpu(cuda):
