@@ -217,8 +217,11 @@ const char* ra_status_string(ra_status status);
 
 /*
  * ra_get_device_error -- synchronises `stream`, then reads and clears this device's error
- * word. Returns RA_OK if no kernel recorded an error since the last call, RA_ERR_TIMEOUT
- * or RA_ERR_DEVICE_BOUNDS if one did, RA_ERR_CUDA if the synchronisation itself failed.
+ * word in one atomic exchange on the device (an error recorded meanwhile by a kernel on
+ * another stream is reported by this call or the next, never lost). Returns RA_OK if no
+ * kernel recorded an error since the last call, RA_ERR_TIMEOUT or RA_ERR_DEVICE_BOUNDS if
+ * one did, RA_ERR_CUDA if the synchronisation or the exchange failed. Calls from several
+ * host threads are serialised.
  */
 ra_status ra_get_device_error(cudaStream_t stream);
 

@@ -105,11 +105,12 @@ def get_device_error(stream=None) -> int:
     return load().ra_get_device_error(_stream_ptr(stream))
 
 
-def selftest_wait_timeout(limit_ns: int = 50_000_000, stream=None) -> int:
+def selftest_wait_timeout(limit_ns: int = 50_000_000, stream=None, read: bool = True) -> int:
     """Launch the failure-detection self-test (a bounded wait that must run out); returns the
-    device error status read afterwards (RA_ERR_TIMEOUT when detection works)."""
+    device error status read afterwards (RA_ERR_TIMEOUT when detection works), or RA_OK
+    without reading when ``read`` is False."""
     _check(load().ra_selftest_wait_timeout(int(limit_ns), _stream_ptr(stream)), "ra_selftest_wait_timeout")
-    return get_device_error(stream)
+    return get_device_error(stream) if read else RA_OK
 
 
 def partial(q, k, v, causal: bool = False, scale: float | None = None,

@@ -180,6 +180,11 @@ ra_status launch_backward(const BwdPlan& pl, ra_dtype dt, int S, cudaStream_t st
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
+// Read and clear the error word in one atomic step: a bit that a kernel on another stream
+// records between a separate read and clear would otherwise be lost.
+__device__ unsigned g_error_snapshot = 0;
+__global__ void take_error_word_kernel() { g_error_snapshot = atomicExch(&g_error_word, 0u); }
+
 ra_status launch_delta(const void* o, const void* d_o, ra_dtype dt, int64_t rows, int d, float* delta,
                        cudaStream_t stream) {
   if (rows == 0) return RA_OK;
@@ -222,13 +227,17 @@ const char* ra_status_string(ra_status s) {
 }
 
 ra_status ra_get_device_error(cudaStream_t stream) {
+  // One host thread at a time: the snapshot variable is shared by all callers of a device.
+  static std::mutex mu;
+  std::lock_guard<std::mutex> g(mu);
   if (cudaStreamSynchronize(stream) != cudaSuccess) return RA_ERR_CUDA;
+  take_error_word_kernel<<<1, 1, 0, stream>>>();
+  if (cudaGetLastError() != cudaSuccess) return RA_ERR_CUDA;
   unsigned word = 0;
-  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return RA_ERR_CUDA;
-  if (word != 0) {
-    const unsigned zero = 0;
-    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return RA_ERR_CUDA;
-  }
+  if (cudaMemcpyFromSymbolAsync(&word, g_error_snapshot, sizeof(word), 0, cudaMemcpyDeviceToHost, stream) !=
+      cudaSuccess)
+    return RA_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return RA_ERR_CUDA;
   if (word & DEVERR_TIMEOUT) return RA_ERR_TIMEOUT;
   if (word & DEVERR_BOUNDS) return RA_ERR_DEVICE_BOUNDS;
   return RA_OK;

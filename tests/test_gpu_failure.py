@@ -21,6 +21,17 @@ def test_wait_timeout_is_reported_and_cleared(cuda):
     assert binding.get_device_error() == binding.RA_OK  # reading clears the word
 
 
+def test_error_recorded_on_one_stream_is_read_on_another(cuda):
+    """The error word belongs to the device: a timeout that a kernel on stream A records is
+    reported by a read on stream B once A has finished, and only once."""
+    a, b = torch.cuda.Stream(), torch.cuda.Stream()
+    assert binding.get_device_error() == binding.RA_OK
+    assert binding.selftest_wait_timeout(20_000_000, stream=a, read=False) == binding.RA_OK
+    a.synchronize()
+    assert binding.get_device_error(b) == binding.RA_ERR_TIMEOUT
+    assert binding.get_device_error(b) == binding.RA_OK
+
+
 def test_context_usable_after_timeout(cuda):
     assert binding.selftest_wait_timeout(20_000_000) == binding.RA_ERR_TIMEOUT
     q, k, v = make_qkv(1, 2, 1024, 128, torch.bfloat16, seed=3, device="cuda")
