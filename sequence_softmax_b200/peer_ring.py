@@ -1,0 +1,254 @@
+"""Ring attention across GPUs with every K/V block read in place from its owner's memory
+(``ring_forward_peer``, ``ring_backward_peer``).
+
+``ring_dist`` moves K||V to the successor at every step with the process group's
+point-to-point calls. GPUs joined by NVLink / NVSwitch can address each other's memory, so
+here no message is sent: each rank maps the other ranks' K||V buffers once (CUDA IPC
+handles, exchanged through the process group) and at step s hands the library the owner's
+pointers for block (rank - s) mod W. The kernels' TMA loads then fetch the tiles from the
+owner's memory as they consume them: the transfer overlaps the compute tile by tile inside
+the kernel, and no copy of a remote block is ever made. Visiting order, causal skip and the
+online-softmax merge are those of ``ring_dist`` ("Ring Attention 논문 분석", listing
+``ring_attention_forward``; gpumode lecture 013 notes, log-sum-exp merge), with the same
+kernels on the same values in the same order, so the two give bit-identical results.
+
+Backward: block c's fp32 dK and dV accumulators live in c's owner's memory. At step s the
+rank holding block (rank - s) mod W adds its queries' contributions into them in place
+(``ra_partial_backward`` stores through the mapped pointers) and into its own dQ. Block c
+is written by rank c + s at step s, so a barrier between steps leaves exactly one writer
+per block at a time, and when the last step ends each owner holds its blocks' dK and dV:
+the listing ``ring_attention_backward``'s reduce, read as that sum, with no return hop.
+
+Only the library's kernels touch another rank's memory (TMA loads without multicast, and
+the backward's accumulator stores); merges, casts and copies run on local buffers.
+Buffers are shared through ``share(tensor, group)`` (default: ``PeerBuffers``), which
+returns an object whose ``views[r]`` is rank r's buffer and whose ``close()`` unmaps them.
+"""
+
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from . import binding
+from .ring_dist import _split_segments, position_segments, ring_schedule, segment_in_future
+
+
+def _cuda_api():
+    try:
+        from cuda.bindings import driver, runtime
+    except ImportError as e:  # pragma: no cover - the image ships cuda-python
+        raise RuntimeError("the peer-memory ring needs cuda-python (cuda.bindings) for CUDA IPC") from e
+    return driver, runtime
+
+
+def _ok(res, what: str):
+    """cuda-python returns (status, outputs...): raise on a failed status, else the outputs."""
+    if int(res[0]) != 0:
+        raise RuntimeError(f"{what} failed: {res[0]}")
+    out = res[1:]
+    return out[0] if len(out) == 1 else out
+
+
+class _DeviceArray:
+    """A raw device pointer in the CUDA array interface, so torch can view it without a copy."""
+
+    def __init__(self, ptr: int, shape, typestr: str):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr, "data": (int(ptr), False),
+                                         "version": 3}
+
+
+# torch dtype -> (array-interface type of the same width, torch dtype of that type)
+_VIEW_TYPES = {torch.bfloat16: ("<i2", torch.int16), torch.float32: ("<f4", torch.float32)}
+
+# Remote allocations mapped by this process: IPC handle bytes -> [device pointer, users].
+# PyTorch's caching allocator can place several tensors in one allocation, whose handles
+# are then identical; each allocation is mapped once and unmapped with its last user.
+_MAPPED: dict = {}
+
+
+def _map(runtime, raw: bytes) -> int:
+    ent = _MAPPED.get(raw)
+    if ent is None:
+        h = runtime.cudaIpcMemHandle_t()
+        h.reserved = raw
+        ptr = _ok(runtime.cudaIpcOpenMemHandle(h, runtime.cudaIpcMemLazyEnablePeerAccess), "cudaIpcOpenMemHandle")
+        ent = _MAPPED[raw] = [int(ptr), 0]
+    ent[1] += 1
+    return ent[0]
+
+
+def _unmap(runtime, raw: bytes):
+    ent = _MAPPED[raw]
+    ent[1] -= 1
+    if ent[1] == 0:
+        del _MAPPED[raw]
+        _ok(runtime.cudaIpcCloseMemHandle(ent[0]), "cudaIpcCloseMemHandle")
+
+
+class PeerBuffers:
+    """Every rank's buffer of one shape and dtype, mapped into this process.
+
+    ``views[r]`` is rank r's buffer (``views[rank]`` is ``local`` itself). The mapping uses
+    legacy CUDA IPC: the handle covers the allocation that holds ``local``, and the offset of
+    ``local`` inside it travels with the handle. ``close()`` unmaps the remote buffers; call
+    it only when no launched kernel reads them any more.
+    """
+
+    def __init__(self, local: torch.Tensor, group=None):
+        if not local.is_cuda or not local.is_contiguous() or local.dtype not in _VIEW_TYPES:
+            raise ValueError("PeerBuffers needs a contiguous CUDA tensor of bf16 or fp32")
+        self.rank = dist.get_rank(group)
+        self._opened = []
+        if dist.get_world_size(group) == 1:
+            self.views = [local]
+            return
+        driver, runtime = _cuda_api()
+        _ok(driver.cuInit(0), "cuInit")
+        base, _size = _ok(driver.cuMemGetAddressRange(local.data_ptr()), "cuMemGetAddressRange")
+        handle = _ok(runtime.cudaIpcGetMemHandle(int(base)), "cudaIpcGetMemHandle")
+        mine = (bytes(handle.reserved), local.data_ptr() - int(base), tuple(local.shape), str(local.dtype))
+        infos = [None] * dist.get_world_size(group)
+        dist.all_gather_object(infos, mine, group=group)
+        typestr, view_dtype = _VIEW_TYPES[local.dtype]
+        self.views = []
+        try:
+            for r, (raw, offset, shape, dtype) in enumerate(infos):
+                if r == self.rank:
+                    self.views.append(local)
+                    continue
+                if shape != tuple(local.shape) or dtype != str(local.dtype):
+                    raise ValueError("every rank must share a buffer of the same shape and dtype")
+                rbase = _map(runtime, raw)
+                self._opened.append(raw)
+                t = torch.as_tensor(_DeviceArray(rbase + offset, shape, typestr), device=local.device)
+                self.views.append(t if view_dtype == local.dtype else t.view(local.dtype))
+        except Exception:
+            self.close()
+            raise
+
+    def close(self):
+        self.views = []
+        opened, self._opened = self._opened, []
+        if opened:
+            _, runtime = _cuda_api()
+            for raw in opened:
+                _unmap(runtime, raw)
+
+
+def _fence(group, device_work: bool):
+    """Every rank's launched work is complete before any rank goes on."""
+    if device_work:
+        torch.cuda.current_stream().synchronize()
+    dist.barrier(group)
+
+
+def _check_local(q_local, others, segs):
+    if sum(s[2] for s in segs) != q_local.shape[2] or any(t.shape != q_local.shape for t in others):
+        raise ValueError("local tensors must hold the N/W tokens of this rank's position")
+
+
+def ring_forward_peer(q_local, k_local, v_local, N: int, layout: str = "contiguous", causal: bool = False,
+                      scale: float | None = None, group=None, kernels=None, share=None):
+    """Exact attention over N tokens split across the ranks of `group`, reading each K/V
+    block from its owner's memory.
+
+    Arguments and result as ``ring_dist.ring_forward_dist``: q_local, k_local, v_local
+    [B, H, N/W, d] on this rank's GPU hold the tokens of virtual position `rank` in
+    increasing token order; returns (O_local in the input dtype, lse_local fp32).
+    ``kernels`` (default: the library binding) provides ``partial`` and ``merge``.
+    """
+    kern = binding if kernels is None else kernels
+    share = PeerBuffers if share is None else share
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    B, H, n_local, d = q_local.shape
+    segs = position_segments(layout, N, world, rank)
+    _check_local(q_local, (k_local, v_local), segs)
+    nseg = len(segs)
+    scale = d ** -0.5 if scale is None else float(scale)
+    dev = q_local.device
+
+    q_s = _split_segments(q_local, nseg)
+    # segment-major, so that each block segment is a contiguous [B, H, L, d] the kernels read in place
+    kv = torch.stack([torch.stack(_split_segments(k_local, nseg)), torch.stack(_split_segments(v_local, nseg))])
+    # per query segment: parts[0] = running state, parts[1] = newest partial
+    state = [(torch.zeros(2, *q.shape, device=dev, dtype=torch.float32),
+              torch.full((2, *q.shape[:3]), float("-inf"), device=dev, dtype=torch.float32)) for q in q_s]
+    peers = share(kv, group)
+    try:
+        _fence(group, kv.is_cuda)  # every rank's K||V is in place before anyone reads it
+        for src in ring_schedule(rank, world):
+            kv_src = peers.views[src]
+            for ki, kseg in enumerate(position_segments(layout, N, world, src)):
+                for qi, qseg in enumerate(segs):
+                    if causal and segment_in_future(qseg, kseg):
+                        continue
+                    parts_o, parts_l = state[qi]
+                    kern.partial(q_s[qi], kv_src[0, ki], kv_src[1, ki], causal=causal, scale=scale, q_tok0=qseg[0],
+                                 q_tok_stride=qseg[1], k_tok0=kseg[0], k_tok_stride=kseg[1], out=parts_o[1],
+                                 lse=parts_l[1])
+                    merged_o, merged_l = kern.merge(parts_o, parts_l, out_dtype=torch.float32)
+                    parts_o[0].copy_(merged_o)
+                    parts_l[0].copy_(merged_l)
+        _fence(group, kv.is_cuda)  # no rank unmaps or frees a buffer another may still read
+    finally:
+        peers.close()
+    out = torch.cat([o[0] for o, _ in state], dim=2).to(q_local.dtype)
+    lse = torch.cat([l[0] for _, l in state], dim=2)
+    return out, lse
+
+
+def ring_backward_peer(q_local, k_local, v_local, o_local, do_local, lse_local, N: int, layout: str = "contiguous",
+                       causal: bool = False, scale: float | None = None, group=None, kernels=None, share=None):
+    """Gradients (dQ, dK, dV) of ``ring_forward_peer``'s output for upstream gradient
+    do_local, every block's dK and dV accumulated in place in its owner's memory.
+
+    Arguments as ``ring_dist.ring_backward_dist`` (lse_local: the forward's final lse);
+    ``kernels`` (default: the library binding) provides ``backward_delta`` and
+    ``partial_backward``. Returns (dQ, dK, dV) [B, H, N/W, d] in the input dtype.
+    """
+    kern = binding if kernels is None else kernels
+    share = PeerBuffers if share is None else share
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    B, H, n_local, d = q_local.shape
+    segs = position_segments(layout, N, world, rank)
+    _check_local(q_local, (k_local, v_local, o_local, do_local), segs)
+    nseg = len(segs)
+    scale = d ** -0.5 if scale is None else float(scale)
+    dev = q_local.device
+
+    delta = kern.backward_delta(o_local, do_local)
+    q_s, do_s = _split_segments(q_local, nseg), _split_segments(do_local, nseg)
+    lse_s, delta_s = _split_segments(lse_local, nseg), _split_segments(delta, nseg)
+    dq_s = [torch.zeros(q.shape, device=dev, dtype=torch.float32) for q in q_s]
+    kv = torch.stack([torch.stack(_split_segments(k_local, nseg)), torch.stack(_split_segments(v_local, nseg))])
+    acc = torch.zeros(kv.shape, device=dev, dtype=torch.float32)  # this rank's blocks' dK, dV
+    peers_kv = share(kv, group)
+    try:
+        peers_acc = share(acc, group)
+    except Exception:
+        peers_kv.close()
+        raise
+    try:
+        _fence(group, kv.is_cuda)
+        for src in ring_schedule(rank, world):
+            kv_src, acc_src = peers_kv.views[src], peers_acc.views[src]
+            for ki, kseg in enumerate(position_segments(layout, N, world, src)):
+                for qi, qseg in enumerate(segs):
+                    if causal and segment_in_future(qseg, kseg):
+                        continue
+                    kern.partial_backward(q_s[qi], kv_src[0, ki], kv_src[1, ki], do_s[qi], lse_s[qi], delta_s[qi],
+                                          dq_s[qi], acc_src[0, ki], acc_src[1, ki], causal=causal, scale=scale,
+                                          q_tok0=qseg[0], q_tok_stride=qseg[1], k_tok0=kseg[0], k_tok_stride=kseg[1])
+            # block src's next writer (rank + 1, next step) starts after these additions
+            _fence(group, kv.is_cuda)
+        own = peers_acc.views[rank]
+        dk = torch.cat(list(own[0]), dim=2).to(k_local.dtype)
+        dv = torch.cat(list(own[1]), dim=2).to(v_local.dtype)
+    finally:
+        peers_acc.close()
+        peers_kv.close()
+    dq = torch.cat(dq_s, dim=2).to(q_local.dtype)
+    return dq, dk, dv
