@@ -235,7 +235,9 @@ ra_status ra_get_device_error(cudaStream_t stream);
  */
 ra_status ra_selftest_wait_timeout(int64_t limit_ns, cudaStream_t stream);
 
-/* ABI version of this header (incremented on any signature change). */
+/* ABI version of this header (incremented on any signature change); ra_abi_version()
+ * returns the version the library was built with, so a caller can compare the two. */
+#define RA_ABI_VERSION 2
 int ra_abi_version(void);
 
 #ifdef __cplusplus

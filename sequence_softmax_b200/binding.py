@@ -20,6 +20,7 @@ library_path = os.environ.get("RA_LIBRARY", os.path.join(_PKG, "libra.so"))
 RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_CUDA, RA_ERR_TIMEOUT, RA_ERR_DEVICE_BOUNDS = range(6)
 RA_F32, RA_BF16 = 0, 1
 LAYOUTS = {"contiguous": 0, "striped": 1, "zigzag": 2}
+ABI_VERSION = 2  # the ABI these signatures describe (ra_abi_version() of a matching library)
 
 # name -> (restype, argtypes) of every symbol include/ra.h declares
 _i64, _i32, _f32, _vp = ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_void_p
@@ -67,6 +68,9 @@ def load():
                 fn = getattr(lib, name)
                 fn.restype = res
                 fn.argtypes = args
+            if lib.ra_abi_version() != ABI_VERSION:
+                raise RuntimeError(f"{library_path} implements ABI {lib.ra_abi_version()}, this binding "
+                                   f"ABI {ABI_VERSION}: rebuild with `python -m sequence_softmax_b200.build`")
             _handle = lib
     return _handle
 

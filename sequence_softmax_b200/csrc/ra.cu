@@ -14,8 +14,6 @@
 #include "bwd_tc.cuh"
 #include "bwd_dq_tc.cuh"
 
-#define RA_ABI_VERSION 2
-
 namespace ra {
 
 // Failure-detection self-test: one thread waits on a barrier that nothing signals, through

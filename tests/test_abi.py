@@ -40,6 +40,9 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_abi_version_and_status_strings(lib):
     assert lib.ra_abi_version() == 2
+    from sequence_softmax_b200 import binding
+    assert binding.ABI_VERSION == lib.ra_abi_version()
+    assert binding.load().ra_abi_version() == binding.ABI_VERSION
     for code in range(6):
         s = binding.status_string(code)
         assert s.startswith("RA_")

@@ -18,7 +18,7 @@ C_PROGRAM = r"""
 #include "ra.h"
 
 int main(void) {
-  if (ra_abi_version() < 1) return 1;
+  if (ra_abi_version() != RA_ABI_VERSION) return 1;
   if (strncmp(ra_status_string(RA_ERR_INVALID_ARG), "RA_ERR_INVALID_ARG", 18) != 0) return 2;
   /* invalid arguments are rejected before any device work */
   if (ra_ring_forward(0, 0, 0, RA_BF16, 1, 1, 256, 128, 0.0f, 2, 1, RA_LAYOUT_ZIGZAG, 0, 0, 0) !=
