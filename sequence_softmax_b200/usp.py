@@ -24,7 +24,7 @@ from __future__ import annotations
 import torch
 import torch.distributed as dist
 
-from . import ring_dist
+from . import peer_ring, ring_dist
 
 
 def usp_groups(R: int, U: int):
@@ -92,23 +92,39 @@ def head_to_seq(y: torch.Tensor, group) -> torch.Tensor:
     return got.movedim(0, 1).reshape(B, U * Hg, S, *rest)
 
 
+def _ring_fns(ring: str):
+    """The inter-group ring: "message" (``ring_dist``: K||V sent each step) or "peer"
+    (``peer_ring``: K/V read in place from the owner's memory)."""
+    if ring == "message":
+        return ring_dist.ring_forward_dist, ring_dist.ring_backward_dist, {}
+    if ring == "peer":
+        return peer_ring.ring_forward_peer, peer_ring.ring_backward_peer, None
+    raise ValueError(f"unknown ring {ring!r}")
+
+
 def usp_forward(q, k, v, N: int, layout: str = "contiguous", causal: bool = False, scale: float | None = None,
-                intra_group=None, inter_group=None, kernels=None):
+                intra_group=None, inter_group=None, kernels=None, ring: str = "message", share=None):
     """Exact attention with the USP split. q, k, v: [B, H, N/(R U), d], this device's tokens
-    (``device_tokens``). Returns (O [B, H, N/(R U), d], lse [B, H, N/(R U)] fp32)."""
+    (``device_tokens``). Returns (O [B, H, N/(R U), d], lse [B, H, N/(R U)] fp32).
+    ``ring`` selects the inter-group ring ("message" or "peer"; ``share`` is passed to the
+    peer ring)."""
+    fwd, _, extra = _ring_fns(ring)
+    extra = {"share": share} if extra is None else extra
     scale = q.shape[-1] ** -0.5 if scale is None else float(scale)
     qh, kh, vh = (seq_to_head(t, intra_group) for t in (q, k, v))
-    o, lse = ring_dist.ring_forward_dist(qh, kh, vh, N, layout, causal, scale, group=inter_group, kernels=kernels)
+    o, lse = fwd(qh, kh, vh, N, layout, causal, scale, group=inter_group, kernels=kernels, **extra)
     return head_to_seq(o, intra_group), head_to_seq(lse, intra_group)
 
 
 def usp_backward(q, k, v, o, d_o, lse, N: int, layout: str = "contiguous", causal: bool = False,
-                 scale: float | None = None, intra_group=None, inter_group=None, kernels=None):
+                 scale: float | None = None, intra_group=None, inter_group=None, kernels=None, ring: str = "message",
+                 share=None):
     """Gradients (dQ, dK, dV) of ``usp_forward``'s output for upstream gradient d_o, all in this
-    device's sequence piece [B, H, N/(R U), d]."""
+    device's sequence piece [B, H, N/(R U), d]. ``ring`` and ``share`` as in ``usp_forward``."""
+    _, bwd, extra = _ring_fns(ring)
+    extra = {"share": share} if extra is None else extra
     scale = q.shape[-1] ** -0.5 if scale is None else float(scale)
     qh, kh, vh, oh, doh = (seq_to_head(t, intra_group) for t in (q, k, v, o, d_o))
     lh = seq_to_head(lse, intra_group)
-    grads = ring_dist.ring_backward_dist(qh, kh, vh, oh, doh, lh, N, layout, causal, scale, group=inter_group,
-                                         kernels=kernels)
+    grads = bwd(qh, kh, vh, oh, doh, lh, N, layout, causal, scale, group=inter_group, kernels=kernels, **extra)
     return tuple(head_to_seq(g, intra_group) for g in grads)

@@ -13,6 +13,8 @@ import torch.multiprocessing as mp
 
 from sequence_softmax_b200 import ring_dist, usp
 
+from .test_peer_ring_host import _SharedPool
+
 
 class _OracleKernels:
     """CPU stand-ins for partial / merge / backward_delta / partial_backward (fp64 oracle)."""
@@ -54,7 +56,7 @@ def _problem(R, U):
     return [r.standard_normal((B, H, N, d)).astype(np.float32) for _ in range(4)]
 
 
-def _main(rank, world, port, R, U, layout, causal, out):
+def _main(rank, world, port, R, U, layout, causal, out, ring="message", pools=None):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
@@ -72,23 +74,37 @@ def _main(rank, world, port, R, U, layout, causal, out):
         hg = (rank % U) * (q.shape[1] // U)
         assert np.array_equal(xh.numpy(), q[:, hg:hg + q.shape[1] // U][:, :, pos])
         assert torch.equal(usp.head_to_seq(xh, intra), x)
+        # peer ring: the ranks of inter group u share pools[u] as their peer memory
+        share = _SharedPool(pools[rank % U]) if ring == "peer" else None
         o, lse = usp.usp_forward(loc(q), loc(k), loc(v), N, layout, causal, intra_group=intra, inter_group=inter,
-                                 kernels=_OracleKernels)
+                                 kernels=_OracleKernels, ring=ring, share=share)
         grads = usp.usp_backward(loc(q), loc(k), loc(v), o, loc(do), lse, N, layout, causal, intra_group=intra,
-                                 inter_group=inter, kernels=_OracleKernels)
+                                 inter_group=inter, kernels=_OracleKernels, ring=ring, share=share)
         out[rank] = (idx, o.numpy(), lse.numpy(), [g.numpy() for g in grads])
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("R,U,layout,causal", [(2, 2, "zigzag", True), (1, 2, "contiguous", True),
-                                               (2, 1, "striped", True), (2, 2, "contiguous", False)])
-def test_usp_matches_definition(R, U, layout, causal):
+@pytest.mark.parametrize("R,U,layout,causal,ring", [(2, 2, "zigzag", True, "message"),
+                                                    (1, 2, "contiguous", True, "message"),
+                                                    (2, 1, "striped", True, "message"),
+                                                    (2, 2, "contiguous", False, "message"),
+                                                    (2, 2, "zigzag", True, "peer"),
+                                                    (3, 1, "striped", True, "peer")])
+def test_usp_matches_definition(R, U, layout, causal, ring):
     import oracle
     world = R * U
+    pools = None
+    if ring == "peer":
+        q, *_ = _problem(R, U)
+        B, H, N, d = q.shape
+        nseg = len(ring_dist.position_segments(layout, N, R, 0))
+        shp = (2, nseg, B, H // U, N // R // nseg, d)
+        # per inter group: share calls forward K||V, backward K||V, backward accumulators
+        pools = [[[torch.zeros(shp).share_memory_() for _ in range(R)] for _ in range(3)] for _ in range(U)]
     out = mp.get_context("spawn").Manager().dict()
-    port = 29900 + 11 * world + 3 * R + os.getpid() % 300
-    mp.spawn(_main, args=(world, port, R, U, layout, causal, out), nprocs=world, join=True)
+    port = 29900 + 11 * world + 3 * R + (50 if ring == "peer" else 0) + os.getpid() % 300
+    mp.spawn(_main, args=(world, port, R, U, layout, causal, out, ring, pools), nprocs=world, join=True)
     q, k, v, do = _problem(R, U)
     d = q.shape[-1]
     o_ref, l_ref = oracle.attention(q, k, v, d ** -0.5, causal)
