@@ -19,8 +19,15 @@ is written by rank c + s at step s, so a barrier between steps leaves exactly on
 per block at a time, and when the last step ends each owner holds its blocks' dK and dV:
 the listing ``ring_attention_backward``'s reduce, read as that sum, with no return hop.
 
-Only the library's kernels touch another rank's memory (TMA loads without multicast, and
-the backward's accumulator stores); merges, casts and copies run on local buffers.
+How K||V is read (``mode``): "direct" hands the kernels the owner's pointers, as above;
+"copy" pulls each step's block one step ahead into a local double buffer with one DMA copy
+(``cudaMemcpyAsync`` on a copy stream), so the block crosses NVLink once while the previous
+step computes and the kernels' re-reads of its tiles (every query tile pair streams the
+whole block) stay in this GPU's L2 and memory instead of crossing NVLink again.
+
+Only the library's kernels and the DMA copies touch another rank's memory (TMA loads
+without multicast, the backward's accumulator stores, ``cudaMemcpyAsync``); merges, casts
+and other copies run on local buffers.
 Buffers are shared through ``share(tensor, group)`` (default: ``PeerBuffers``), which
 returns an object whose ``views[r]`` is rank r's buffer and whose ``close()`` unmaps them.
 """
@@ -143,20 +150,79 @@ def _fence(group, device_work: bool):
     dist.barrier(group)
 
 
+class _Blocks:
+    """The K||V block of each ring step, as the tensor this rank's kernels read.
+
+    "direct": the owner's buffer itself; the kernels' TMA loads fetch every tile they read
+    over NVLink, including the re-reads (each query tile pair streams the whole block).
+    "copy": a local double buffer. While step s computes, the block of step s + 1 is pulled
+    from its owner with one DMA copy (``cudaMemcpyAsync``) on a copy stream, so each block
+    crosses NVLink once, the transfer overlaps the compute, and the re-reads hit this GPU's
+    L2 and memory. Call ``get(s)`` and ``done(s)`` in step order.
+    """
+
+    def __init__(self, mode: str, peers, sched, local_kv: torch.Tensor):
+        if mode not in ("direct", "copy"):
+            raise ValueError(f"unknown mode {mode!r}")
+        self.mode, self.peers, self.sched = mode, peers, sched
+        self.cuda = local_kv.is_cuda
+        if mode == "copy" and len(sched) > 1:
+            self.bufs = [torch.empty_like(local_kv) for _ in range(2)]
+            self.copy_stream = torch.cuda.Stream(device=local_kv.device) if self.cuda else None
+            self.ready = [None, None]  # copy into bufs[i] complete
+            self.freed = [None, None]  # the kernels that read bufs[i] complete
+
+    def get(self, s: int) -> torch.Tensor:
+        """Block of step s; in "copy" mode also starts the pull of step s + 1's block."""
+        if self.mode == "direct":
+            return self.peers.views[self.sched[s]]
+        if s + 1 < len(self.sched):
+            self._pull((s + 1) % 2, self.peers.views[self.sched[s + 1]])
+        if s == 0:
+            return self.peers.views[self.sched[0]]  # this rank's own block
+        if self.cuda:
+            torch.cuda.current_stream().wait_event(self.ready[s % 2])
+        return self.bufs[s % 2]
+
+    def done(self, s: int):
+        """Step s's kernels are enqueued; the buffer they read may be refilled after them."""
+        if self.mode == "copy" and s > 0 and self.cuda:
+            ev = torch.cuda.Event()
+            ev.record(torch.cuda.current_stream())
+            self.freed[s % 2] = ev
+
+    def _pull(self, i: int, src: torch.Tensor):
+        dst = self.bufs[i]
+        if not self.cuda:
+            dst.copy_(src)
+            return
+        if self.freed[i] is not None:
+            self.copy_stream.wait_event(self.freed[i])
+        _, runtime = _cuda_api()
+        _ok(runtime.cudaMemcpyAsync(dst.data_ptr(), src.data_ptr(), dst.numel() * dst.element_size(),
+                                    runtime.cudaMemcpyKind.cudaMemcpyDeviceToDevice,
+                                    runtime.cudaStream_t(self.copy_stream.cuda_stream)), "cudaMemcpyAsync")
+        ev = torch.cuda.Event()
+        ev.record(self.copy_stream)
+        self.ready[i] = ev
+
+
 def _check_local(q_local, others, segs):
     if sum(s[2] for s in segs) != q_local.shape[2] or any(t.shape != q_local.shape for t in others):
         raise ValueError("local tensors must hold the N/W tokens of this rank's position")
 
 
 def ring_forward_peer(q_local, k_local, v_local, N: int, layout: str = "contiguous", causal: bool = False,
-                      scale: float | None = None, group=None, kernels=None, share=None):
+                      scale: float | None = None, group=None, kernels=None, share=None, mode: str = "direct"):
     """Exact attention over N tokens split across the ranks of `group`, reading each K/V
     block from its owner's memory.
 
     Arguments and result as ``ring_dist.ring_forward_dist``: q_local, k_local, v_local
     [B, H, N/W, d] on this rank's GPU hold the tokens of virtual position `rank` in
     increasing token order; returns (O_local in the input dtype, lse_local fp32).
-    ``kernels`` (default: the library binding) provides ``partial`` and ``merge``.
+    ``kernels`` (default: the library binding) provides ``partial`` and ``merge``. ``mode``:
+    "direct" (the kernels read the owner's buffer) or "copy" (each block pulled into a local
+    buffer one step ahead; see ``_Blocks``).
     """
     kern = binding if kernels is None else kernels
     share = PeerBuffers if share is None else share
@@ -177,9 +243,11 @@ def ring_forward_peer(q_local, k_local, v_local, N: int, layout: str = "contiguo
               torch.full((2, *q.shape[:3]), float("-inf"), device=dev, dtype=torch.float32)) for q in q_s]
     peers = share(kv, group)
     try:
+        sched = ring_schedule(rank, world)
+        blocks = _Blocks(mode, peers, sched, kv)
         _fence(group, kv.is_cuda)  # every rank's K||V is in place before anyone reads it
-        for src in ring_schedule(rank, world):
-            kv_src = peers.views[src]
+        for s, src in enumerate(sched):
+            kv_src = blocks.get(s)
             for ki, kseg in enumerate(position_segments(layout, N, world, src)):
                 for qi, qseg in enumerate(segs):
                     if causal and segment_in_future(qseg, kseg):
@@ -191,6 +259,7 @@ def ring_forward_peer(q_local, k_local, v_local, N: int, layout: str = "contiguo
                     merged_o, merged_l = kern.merge(parts_o, parts_l, out_dtype=torch.float32)
                     parts_o[0].copy_(merged_o)
                     parts_l[0].copy_(merged_l)
+            blocks.done(s)
         _fence(group, kv.is_cuda)  # no rank unmaps or frees a buffer another may still read
     finally:
         peers.close()
@@ -200,13 +269,16 @@ def ring_forward_peer(q_local, k_local, v_local, N: int, layout: str = "contiguo
 
 
 def ring_backward_peer(q_local, k_local, v_local, o_local, do_local, lse_local, N: int, layout: str = "contiguous",
-                       causal: bool = False, scale: float | None = None, group=None, kernels=None, share=None):
+                       causal: bool = False, scale: float | None = None, group=None, kernels=None, share=None,
+                       mode: str = "direct"):
     """Gradients (dQ, dK, dV) of ``ring_forward_peer``'s output for upstream gradient
     do_local, every block's dK and dV accumulated in place in its owner's memory.
 
     Arguments as ``ring_dist.ring_backward_dist`` (lse_local: the forward's final lse);
     ``kernels`` (default: the library binding) provides ``backward_delta`` and
-    ``partial_backward``. Returns (dQ, dK, dV) [B, H, N/W, d] in the input dtype.
+    ``partial_backward``. ``mode`` chooses how K||V is read, as in ``ring_forward_peer``; the
+    dK and dV accumulators are always added into in the owner's memory (each key tile's
+    sums are stored once per step). Returns (dQ, dK, dV) [B, H, N/W, d] in the input dtype.
     """
     kern = binding if kernels is None else kernels
     share = PeerBuffers if share is None else share
@@ -232,9 +304,11 @@ def ring_backward_peer(q_local, k_local, v_local, o_local, do_local, lse_local, 
         peers_kv.close()
         raise
     try:
+        sched = ring_schedule(rank, world)
+        blocks = _Blocks(mode, peers_kv, sched, kv)
         _fence(group, kv.is_cuda)
-        for src in ring_schedule(rank, world):
-            kv_src, acc_src = peers_kv.views[src], peers_acc.views[src]
+        for s, src in enumerate(sched):
+            kv_src, acc_src = blocks.get(s), peers_acc.views[src]
             for ki, kseg in enumerate(position_segments(layout, N, world, src)):
                 for qi, qseg in enumerate(segs):
                     if causal and segment_in_future(qseg, kseg):
@@ -242,6 +316,7 @@ def ring_backward_peer(q_local, k_local, v_local, o_local, do_local, lse_local, 
                     kern.partial_backward(q_s[qi], kv_src[0, ki], kv_src[1, ki], do_s[qi], lse_s[qi], delta_s[qi],
                                           dq_s[qi], acc_src[0, ki], acc_src[1, ki], causal=causal, scale=scale,
                                           q_tok0=qseg[0], q_tok_stride=qseg[1], k_tok0=kseg[0], k_tok_stride=kseg[1])
+            blocks.done(s)
             # block src's next writer (rank + 1, next step) starts after these additions
             _fence(group, kv.is_cuda)
         own = peers_acc.views[rank]

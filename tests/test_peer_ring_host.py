@@ -74,7 +74,7 @@ def _inputs(world, causal):
     return (B, H, N, d), q, k, v, do, o, lse
 
 
-def _main(rank, world, port, layout, causal, pool, out):
+def _main(rank, world, port, layout, causal, pool, out, mode="direct"):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
@@ -83,17 +83,19 @@ def _main(rank, world, port, layout, causal, pool, out):
         loc = lambda x: torch.from_numpy(np.ascontiguousarray(x[:, :, idx])).float()  # noqa: E731
         share = _SharedPool(pool)
         of, lf = peer_ring.ring_forward_peer(loc(q), loc(k), loc(v), N, layout, causal, kernels=_OracleForwardKernels,
-                                             share=share)
+                                             share=share, mode=mode)
         g = peer_ring.ring_backward_peer(loc(q), loc(k), loc(v), loc(o), loc(do), loc(lse), N, layout, causal,
-                                         kernels=_OracleKernels, share=share)
+                                         kernels=_OracleKernels, share=share, mode=mode)
         out[rank] = (idx, of.numpy(), lf.numpy(), [t.numpy() for t in g])
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,layout,causal", [(2, "contiguous", True), (3, "zigzag", True), (2, "striped", True),
-                                                 (3, "contiguous", False)])
-def test_peer_ring_forward_and_backward(world, layout, causal):
+@pytest.mark.parametrize("world,layout,causal,mode", [(2, "contiguous", True, "direct"), (3, "zigzag", True, "direct"),
+                                                      (2, "striped", True, "direct"), (3, "contiguous", False, "direct"),
+                                                      (3, "zigzag", True, "copy"), (2, "striped", True, "copy"),
+                                                      (4, "contiguous", False, "copy")])
+def test_peer_ring_forward_and_backward(world, layout, causal, mode):
     """Every rank's O, lse, dQ, dK and dV equal the definition's for its tokens."""
     import oracle
     (B, H, N, d), q, k, v, do, o, lse = _inputs(world, causal)
@@ -101,8 +103,8 @@ def test_peer_ring_forward_and_backward(world, layout, causal):
     # share calls in order: forward K||V, backward K||V, backward dK||dV accumulators
     pool = [[torch.zeros(shp).share_memory_() for _ in range(world)] for _ in range(3)]
     out = mp.get_context("spawn").Manager().dict()
-    port = 29550 + 5 * world + os.getpid() % 400
-    mp.spawn(_main, args=(world, port, layout, causal, pool, out), nprocs=world, join=True)
+    port = 29550 + 5 * world + (2 if mode == "copy" else 0) + os.getpid() % 400
+    mp.spawn(_main, args=(world, port, layout, causal, pool, out, mode), nprocs=world, join=True)
     ref = oracle.attention_backward(q, k, v, do, d ** -0.5, causal)
     for rk in range(world):
         idx, of, lf, got = out[rk]
