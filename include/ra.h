@@ -19,11 +19,16 @@
  * Conventions shared by every entry point
  *   - Pointers are device pointers owned by the caller, contiguous, 16-byte aligned.
  *     Tensors are row-major [B, H, rows, d] with d innermost (the head dimension).
+ *     ra_partial's k, v and ra_partial_backward's k, v, dk_acc, dv_acc may address another
+ *     GPU's memory mapped into this process (CUDA IPC with peer access): the kernels read
+ *     it with TMA loads that never use cluster multicast and write it with plain stores.
  *   - Calls are asynchronous on `stream`. The return value reports argument and launch
  *     errors only; nothing has been launched when it is not RA_OK. Errors found on the
  *     device (a bounded wait that ran out) are reported by ra_get_device_error().
- *   - The library allocates no device memory. Its only device state is one 32-bit error
- *     word per device, a static variable of the library image.
+ *   - The library allocates no device memory. Its only device state is static variables of
+ *     the library image, per device: the 32-bit error word (and the copy that
+ *     ra_get_device_error reads it through) and the scratch array of
+ *     ra_ring_backward_noalloc.
  *   - scale is the softmax scale, normally d^-1/2 ([BLOG] blockwise_attention; [GLOSSARY]).
  *   - Causal masking keeps key token j for query token i iff j <= i: the diagonal is kept
  *     ([BLOG] ring_attention_causal_step masks triu(diagonal=1)).
