@@ -1,6 +1,5 @@
 """The backward oracle against its pins, and planted mistakes that some pin must catch."""
 
-import numpy as np
 import pytest
 
 from oracle import backward as Bk
