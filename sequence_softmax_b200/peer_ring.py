@@ -96,7 +96,8 @@ def _unmap(runtime, raw: bytes):
 class PeerBuffers:
     """Every rank's buffer of one shape and dtype, mapped into this process.
 
-    ``views[r]`` is rank r's buffer (``views[rank]`` is ``local`` itself). The mapping uses
+    ``views[r]`` is rank r's buffer (``views[rank]`` is ``local`` itself); a remote view's
+    torch device may name the owner's GPU, and only its pointer is meant to be used. The mapping uses
     legacy CUDA IPC: the handle covers the allocation that holds ``local``, and the offset of
     ``local`` inside it travels with the handle. ``close()`` unmaps the remote buffers; call
     it only when no launched kernel reads them any more.
@@ -128,7 +129,12 @@ class PeerBuffers:
                     raise ValueError("every rank must share a buffer of the same shape and dtype")
                 rbase = _map(runtime, raw)
                 self._opened.append(raw)
-                t = torch.as_tensor(_DeviceArray(rbase + offset, shape, typestr), device=local.device)
+                # No device argument: torch takes the device from the pointer (possibly the
+                # owner's GPU) and never copies. The view is only handed to the library and to
+                # DMA copies as a pointer; no torch operation that launches a kernel touches it.
+                t = torch.as_tensor(_DeviceArray(rbase + offset, shape, typestr))
+                if t.data_ptr() != rbase + offset:
+                    raise RuntimeError("a peer buffer view must alias the mapped memory")
                 self.views.append(t if view_dtype == local.dtype else t.view(local.dtype))
         except Exception:
             self.close()
