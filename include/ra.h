@@ -21,7 +21,8 @@
  *     Tensors are row-major [B, H, rows, d] with d innermost (the head dimension).
  *     ra_partial's k, v and ra_partial_backward's k, v, dk_acc, dv_acc may address another
  *     GPU's memory mapped into this process (CUDA IPC with peer access): the kernels read
- *     it with TMA loads that never use cluster multicast and write it with plain stores.
+ *     it with plain per-CTA TMA loads (each CTA fetches its own tiles) and writes it with
+ *     plain stores.
  *   - Calls are asynchronous on `stream`. The return value reports argument and launch
  *     errors only; nothing has been launched when it is not RA_OK. Errors found on the
  *     device (a bounded wait that ran out) are reported by ra_get_device_error().
@@ -202,13 +203,16 @@ ra_status ra_ring_backward(const void* q, const void* k, const void* v, const vo
  * it until the process exits. Problems whose ra_ring_backward_workspace_bytes() exceeds it
  * (B*H*N > 16777216 rows) return RA_ERR_UNSUPPORTED without launching anything.
  *
- * The first call on a device looks up the array's device address, with that device current,
- * and keeps it; make that first call before any stream capture. All calls on a device share
- * the one array: two calls whose work overlaps on the GPU (different streams, or different
- * host threads without ordering) race on it and corrupt each other's gradients, so order
- * them on one stream or synchronise between them. Nothing needs clearing by the caller: each
- * call zeroes the part of the array that must start at zero. Arguments, layouts and outputs
- * are those of ra_ring_backward.
+ * The first call on a device (in a given CUDA context) looks up the array's device address,
+ * with that device current, and keeps it; make that first call before any stream capture.
+ * A later call from another context on the same device (after cudaDeviceReset, or with a
+ * different context made current through the driver API) looks the address up again. All
+ * calls on a device share the one array: two calls whose work overlaps on the GPU
+ * (different streams, or different host threads without ordering) race on it and corrupt
+ * each other's gradients, so order them on one stream or synchronise between them. Nothing
+ * needs clearing: every call overwrites each scratch entry it reads (the row term of each of
+ * its B*H*N query rows) before reading it, so what an earlier call left there never matters.
+ * Arguments, layouts and outputs are those of ra_ring_backward.
  */
 #define RA_NOALLOC_SCRATCH_BYTES (64ll * 1024 * 1024)
 ra_status ra_ring_backward_noalloc(const void* q, const void* k, const void* v, const void* o,

@@ -433,19 +433,46 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[RA_NOALLOC_SCRA
 
 namespace {
 
+// cuCtxGetCurrent through the runtime's driver entry point (no -lcuda).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
 // Device address of this device's copy of g_noalloc_scratch (host code only sees a
-// host-side stand-in for the name). Looked up once per device, with that device current.
+// host-side stand-in for the name). Looked up with the device current, once per device and
+// CUDA context: the address belongs to the context the library's module is loaded in, so a
+// new context on the device (after cudaDeviceReset, or another context made current) gets
+// a fresh lookup instead of a stale address.
 ra_status noalloc_scratch(void** out) {
   static void* addr[64] = {};
+  static CUcontext owner[64] = {};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return RA_ERR_CUDA;
   if (dev < 0 || dev >= 64) return RA_ERR_UNSUPPORTED;
+  CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+  CUcontext ctx = nullptr;
+  if (!get_ctx || get_ctx(&ctx) != CUDA_SUCCESS) return RA_ERR_CUDA;
   std::lock_guard<std::mutex> g(mu);
-  if (addr[dev] == nullptr) {
+  // No context current yet (nothing has touched this device): the lookup binds the
+  // runtime's context, which is then recorded as the owner.
+  if (ctx == nullptr || addr[dev] == nullptr || owner[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return RA_ERR_CUDA;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return RA_ERR_CUDA;
     addr[dev] = p;
+    owner[dev] = ctx;
   }
   *out = addr[dev];
   return RA_OK;
