@@ -188,7 +188,7 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   return true;
 }
 
-// 4-D tiled TMA load of one box into shared memory, completing on `bar` (no multicast).
+// 4-D tiled TMA load of one box into this CTA's shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int c0, int c1, int c2, int c3) {
   asm volatile(

@@ -25,8 +25,8 @@ How K||V is read (``mode``): "direct" hands the kernels the owner's pointers, as
 step computes and the kernels' re-reads of its tiles (every query tile pair streams the
 whole block) stay in this GPU's L2 and memory instead of crossing NVLink again.
 
-Only the library's kernels and the DMA copies touch another rank's memory (TMA loads
-without multicast, the backward's accumulator stores, ``cudaMemcpyAsync``); merges, casts
+Only the library's kernels and the DMA copies touch another rank's memory (plain per-CTA
+TMA loads, the backward's accumulator stores, ``cudaMemcpyAsync``); merges, casts
 and other copies run on local buffers.
 Buffers are shared through ``share(tensor, group)`` (default: ``PeerBuffers``), which
 returns an object whose ``views[r]`` is rank r's buffer and whose ``close()`` unmaps them.
