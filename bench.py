@@ -9,15 +9,27 @@ the call is one kernel launch that runs every step of the path (layout walk, Q/K
 QK^T, causal predicate, online softmax, PV, finalise). Inputs are synthetic (seeded i.i.d.
 N(0, 1)), resident in HBM and 6.4 GB in total, so they exceed the 126 MB L2 between steps.
 
-Rank 0 prints one JSON line. With N > 1 (torchrun) every rank runs an independent replica
-of the workload with its own seed (weak scaling, no collective on the data path); time is
-the max over ranks of CUDA-event time.
+Rank 0 prints one JSON line. With N > 1 (torchrun), the default (--multi ring) runs the
+pages' own partition of the same workload over the N GPUs: each rank holds the tokens of one
+virtual ring position (zig-zag: chunks r and 2N-1-r), keeps its queries, and K||V rotates
+around the ring over NCCL while ra_partial + ra_merge fold each block into the running state
+("Ring Attention 논문 분석", listing ring_attention_forward). The total work is fixed (strong
+scaling). --multi replicas instead runs an independent replica of the workload per rank
+(weak scaling, no collective on the data path). Time is the max over ranks of CUDA-event
+time.
 
 Sub-measurements in the same line: "merge" (ra_merge, HBM-bound) and "backward"
 (ra_ring_backward on the 128K-token zig-zag workload).
 
 --impl reference times the fp64 CPU oracle on this host's cores on a bounded sample of the
 same workload (rows of one head against all their visible keys) in the same unit.
+
+--report prints one JSON line per named workload (the toy, 4K non-causal and its Q x 4
+variant, 32K causal, 128K zig-zag and striped, 1M zig-zag) and per merge workload (n = 2 and
+n = 16 partial states): device time, TFLOP/s (or GB/s) and roofline fractions, clocks, the
+error against the fp64 oracle (every row on the small workloads, sampled rows on the long
+ones) and the oracle's CPU time (measured in full on the small workloads, measured on the
+sampled rows and extrapolated by visible pairs on the long ones).
 """
 
 from __future__ import annotations
@@ -66,6 +78,11 @@ def parse():
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--bwd-workload", default=BWD_WORKLOAD)
     ap.add_argument("--bwd-steps", type=int, default=3)
+    ap.add_argument("--multi", choices=["ring", "replicas"], default="ring",
+                    help="with N > 1 GPUs: the ring over NCCL (one virtual position per rank) or replicas")
+    ap.add_argument("--report", action="store_true", help="one JSON line per named workload (see the docstring)")
+    ap.add_argument("--report-rows", type=int, default=512,
+                    help="sampled query rows per head checked against the oracle on the long workloads")
     return ap.parse_args()
 
 
@@ -161,14 +178,29 @@ class ClockSampler:
 # CPU oracle sample (the reference arm and the cpu_baseline of the GPU arm).
 # ------------------------------------------------------------------------------------------
 
-def oracle_sample(w, seconds: float, seed: int = 0):
-    """Times the fp64 oracle on query rows of one head until ~`seconds` of CPU work.
+ORACLE_ROWS_PER_CALL = 256  # query rows per oracle call: one fixed sample size for both arms
 
-    Returns (tflops, elapsed_s, n_rows, threads). Work is counted with the same rule as the
-    GPU metric: 4 d FLOPs per visible (query, key) pair.
+
+def blas_threads() -> int:
+    """Host threads the oracle's BLAS runs on: the cores this process may use."""
+    return cpu_cores()
+
+
+def oracle_sample(w, calls: int = 0, seconds: float = 0.0, seed: int = 0):
+    """Times the fp64 oracle, as it stands, on fixed-size samples of one head's query rows.
+
+    Every call evaluates ORACLE_ROWS_PER_CALL random query rows against all their visible
+    keys (``oracle.attention`` with its default row blocks), so its fixed per-call cost
+    (widening the head's K and V to fp64) is amortised the same way in every measurement.
+    Runs ``calls`` calls, or as many as fill ``seconds``. BLAS threads are pinned to the
+    cores this process may use. Work is counted with the GPU metric's rule: 4 d FLOPs per
+    visible (query, key) pair.
+
+    Returns (tflops, elapsed_s, n_rows, threads, n_calls).
     """
     import numpy as np
     import torch
+    from threadpoolctl import threadpool_limits
 
     import oracle
     from sequence_softmax_b200.inputs import make_qkv
@@ -176,20 +208,20 @@ def oracle_sample(w, seconds: float, seed: int = 0):
     g = torch.Generator().manual_seed(1000 + seed)
     q, k, v = make_qkv(1, 1, w.N, w.d, w.torch_dtype, seed=w.seed, device="cpu", q_scale=w.q_scale)
     qn, kn, vn = (t.float().numpy() for t in (q, k, v))
-    threads = torch.get_num_threads()
-    done_flops, t_total, rows_done = 0, 0.0, 0
-    batch = 8
-    while t_total < seconds:
-        rows = torch.randint(0, w.N, (batch,), generator=g).numpy()
-        t0 = time.perf_counter()
-        oracle.attention(qn, kn, vn, w.scale, w.causal, rows=rows, row_block=batch)
-        t_total += time.perf_counter() - t0
-        vis = (rows + 1) if w.causal else np.full(batch, w.N)
-        done_flops += int(4 * w.d * vis.sum())
-        rows_done += batch
-        if t_total < seconds / 4:
-            batch = min(batch * 2, 256)
-    return done_flops / t_total / 1e12, t_total, rows_done, threads
+    threads = blas_threads()
+    done_flops, t_total, rows_done, n = 0, 0.0, 0, 0
+    R = min(ORACLE_ROWS_PER_CALL, w.N)
+    with threadpool_limits(limits=threads):
+        while (calls and n < calls) or (not calls and (t_total < seconds or n == 0)):
+            rows = torch.randint(0, w.N, (R,), generator=g).numpy()
+            t0 = time.perf_counter()
+            oracle.attention(qn, kn, vn, w.scale, w.causal, rows=rows)
+            t_total += time.perf_counter() - t0
+            vis = (rows + 1) if w.causal else np.full(R, w.N)
+            done_flops += int(4 * w.d * vis.sum())
+            rows_done += R
+            n += 1
+    return done_flops / t_total / 1e12, t_total, rows_done, threads, n
 
 
 def cpu_cores():
@@ -200,28 +232,23 @@ def cpu_cores():
 
 
 def run_reference(a, w):
+    """The reference arm: the fp64 oracle on this host's cores, one fixed-size sample of the
+    workload per step (rank 0 only; other ranks exit without work)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    per_step = max(2.0, min(a.cpu_seconds, 20.0) / max(1, a.steps))
-    for _ in range(a.warmup):
-        oracle_sample(w, min(1.0, per_step))
-    vals, secs, rows = [], 0.0, 0
-    for s in range(a.steps):
-        tf, el, nr, threads = oracle_sample(w, per_step, seed=s + 1)
-        vals.append(tf)
-        secs += el
-        rows += nr
-    value = statistics.mean(vals)
+    oracle_sample(w, calls=a.warmup, seed=0)
+    tf, secs, rows, threads, n = oracle_sample(w, calls=a.steps, seed=1)
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": a.gpus,
+        "impl": "reference", "metric": METRIC, "value": tf, "unit": "TFLOP/s", "n_gpus": a.gpus,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": secs / a.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w),
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                         "sample": f"{rows} query rows of head 0 against all their visible keys "
-                                   f"(fp64 NumPy oracle), {secs:.1f} s total"},
-        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "cpu_baseline": {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{n} calls x {ORACLE_ROWS_PER_CALL} random query rows of head 0 against all "
+                                   f"their visible keys (fp64 NumPy oracle, BLAS pinned to {threads} threads), "
+                                   f"{secs:.1f} s total"},
+        "e2e": {"value": tf, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
     print(json.dumps(line), flush=True)
@@ -254,7 +281,15 @@ def main():
     w = WORKLOADS[a.workload or BENCH_WORKLOAD]
     if a.impl == "reference":
         return run_reference(a, w)
+    if a.report:
+        return run_report(a)
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1 and a.multi == "ring":
+        return run_ring(a, w)
+    return run_single(a, w)
 
+
+def run_single(a, w):
+    """One ra_ring_forward call per step on each rank's own replica of the workload."""
     import torch
     import torch.distributed as dist
 
@@ -311,7 +346,8 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": workload_config(w),
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(w), parallelism=f"replicas{world}" if world > 1 else "single"),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{pk['source']} bf16 burst",
@@ -336,10 +372,11 @@ def main():
         torch.cuda.empty_cache()
 
     if rank == 0 and not a.no_cpu_baseline and world == 1:
-        tf, el, nr, threads = oracle_sample(w, a.cpu_seconds)
+        tf, el, nr, threads, n = oracle_sample(w, seconds=a.cpu_seconds)
         line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                                "sample": f"{nr} random query rows of head 0 against all their visible keys, "
-                                          f"fp64 NumPy oracle, {el:.1f} s (host has {cpu_cores()} cores)"}
+                                "sample": f"{n} calls x {ORACLE_ROWS_PER_CALL} random query rows of head 0 against "
+                                          f"all their visible keys, fp64 NumPy oracle, BLAS pinned to {threads} "
+                                          f"threads, {el:.1f} s"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -433,7 +470,7 @@ def bench_e2e(binding, torch, w, q, k, v, world, a):
     qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
     oh = torch.empty(qh.shape, dtype=qh.dtype, pin_memory=True)
     lh = torch.empty(w.B, w.H, w.N, dtype=torch.float32, pin_memory=True)
-    steps = max(1, min(a.steps, 3))
+    steps = a.steps
     binding.ring_forward(qh, kh, vh, w.n_chunks, w.causal, w.layout, out=oh, lse=lh)  # warm
     torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -447,6 +484,277 @@ def bench_e2e(binding, torch, w, q, k, v, world, a):
     d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
     return {"value": world * w.flops() / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+# ------------------------------------------------------------------------------------------
+# N > 1: the ring across GPUs.
+# ------------------------------------------------------------------------------------------
+
+def position_tokens(t, segs):
+    """The tokens of one virtual ring position (segments (tok0, stride, count)) of a
+    [B, H, N, d] tensor, in increasing token order: [B, H, N / W, d], contiguous."""
+    import torch
+    return torch.cat([t[:, :, t0:t0 + stride * n:stride] for (t0, stride, n) in segs], dim=2).contiguous()
+
+
+class CountingKernels:
+    """The binding's entry points, counting the library launches made through them."""
+
+    def __init__(self, binding):
+        self._binding = binding
+        self.launches = 0
+
+    def __getattr__(self, name):
+        fn = getattr(self._binding, name)
+
+        def call(*args, **kwargs):
+            self.launches += 1  # partial, merge: one kernel launch per call
+            return fn(*args, **kwargs)
+        return call
+
+
+def run_ring(a, w):
+    """The workload's attention over the N ranks as the pages partition it: rank r holds the
+    tokens of virtual position r (the workload's layout over N positions), keeps its queries,
+    and K||V rotates around the ring over NCCL (ring_dist.ring_forward_dist). The total work
+    is the workload's (strong scaling)."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from sequence_softmax_b200 import binding
+    from sequence_softmax_b200.inputs import workload_qkv
+    from sequence_softmax_b200.ring_dist import position_segments, ring_forward_dist
+
+    world = int(os.environ["WORLD_SIZE"])
+    rank = int(os.environ["RANK"])
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    pk = peaks()
+
+    # The whole problem, drawn identically on every rank; each rank keeps its position's tokens.
+    q, k, v = workload_qkv(w, device=dev)
+    segs = position_segments(w.layout, w.N, world, rank)
+    ql, kl, vl = (position_tokens(t, segs) for t in (q, k, v))
+    del q, k, v
+    torch.cuda.empty_cache()
+    kern = CountingKernels(binding)
+
+    def step():
+        return ring_forward_dist(ql, kl, vl, w.N, w.layout, w.causal, kernels=kern)
+
+    for _ in range(a.warmup):
+        step()
+    torch.cuda.synchronize()
+    if binding.get_device_error() != binding.RA_OK:
+        raise RuntimeError("device error during warm-up")
+    stream = torch.cuda.current_stream()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    kern.launches = 0
+    with ClockSampler(local) as clk:
+        dist.barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for _ in range(a.steps):
+            step()
+        end.record(stream)
+        dist.barrier()
+        torch.cuda.synchronize()
+    ms = max_over_ranks(start.elapsed_time(end), world, dev)
+    launches = torch.tensor([kern.launches], device=dev, dtype=torch.int64)
+    dist.all_reduce(launches)
+    if binding.get_device_error() != binding.RA_OK:
+        raise RuntimeError("device error during the timed region")
+    ms_step = ms / a.steps
+    flops = w.flops()
+    value = flops / (ms_step / 1e3) / 1e12
+    per_gpu = value / world
+    peak = pk["bf16_tflops"]
+    cfg = dict(workload_config(w), n_chunks=world, parallelism=f"ring{world}",
+               partition=f"rank r holds virtual position r of {world} ({w.layout}); K||V rotates over NCCL")
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+        "roofline": {"bound": "tensor", "achieved": per_gpu, "peak": peak, "unit": "TFLOP/s",
+                     "frac": per_gpu / peak, "traffic": None, "peak_source": f"{pk['source']} bf16 burst",
+                     "note": "per-GPU step throughput of the ring (ra_partial's attn_fwd_tc_kernel<128> "
+                             "launches plus ra_merge and the exchange), not one launch",
+                     "kernel": "attn_fwd_tc_kernel<128> via ra_partial"},
+        "clocks": clk.summary(),
+        "gpu_launches": int(launches.item()),
+    }
+    if not a.no_e2e:
+        qh, kh, vh = (t.cpu().pin_memory() for t in (ql, kl, vl))
+        qd, kd, vd = torch.empty_like(ql), torch.empty_like(kl), torch.empty_like(vl)
+        oh = torch.empty(qh.shape, dtype=qh.dtype, pin_memory=True)
+        lh = torch.empty(qh.shape[:3], dtype=torch.float32, pin_memory=True)
+
+        def e2e_step():
+            for d_, h_ in ((qd, qh), (kd, kh), (vd, vh)):
+                d_.copy_(h_, non_blocking=True)
+            o, l = ring_forward_dist(qd, kd, vd, w.N, w.layout, w.causal)
+            oh.copy_(o, non_blocking=True)
+            lh.copy_(l, non_blocking=True)
+
+        e2e_step()
+        dist.barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for _ in range(a.steps):
+            e2e_step()
+        end.record(stream)
+        dist.barrier()
+        torch.cuda.synchronize()
+        ems = max_over_ranks(start.elapsed_time(end), world, dev) / a.steps
+        h2d = world * sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+        d2h = world * (oh.numel() * oh.element_size() + lh.numel() * lh.element_size())
+        line["e2e"] = {"value": flops / (ems / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ems,
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": a.steps,
+                       "note": "bytes summed over all ranks"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------------------------------
+# --report: one line per named workload.
+# ------------------------------------------------------------------------------------------
+
+REPORT_WORKLOADS = ["toy-4dev-seq32-d16", "seq4k-d64-noncausal-8chunks", "seq4k-d64-noncausal-8chunks-qx4",
+                    "seq32k-d128-causal-contig8", "seq128k-d128-causal-zigzag16", "seq128k-d128-causal-striped16",
+                    "seq1m-d128-causal-zigzag16"]
+REPORT_MERGES = [(2, 8 * (1 << 20), 128), (16, 32 * (1 << 17), 128)]
+L2_FLUSH_BYTES = 256 << 20  # written between timed iterations: twice the 126 MB L2
+
+
+def _time_each(fn, n_iter, flush, stream, torch):
+    """Median CUDA-event time of fn over n_iter iterations, L2 flushed before each."""
+    times = []
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(n_iter):
+        flush.zero_()
+        s.record(stream)
+        fn()
+        e.record(stream)
+        e.synchronize()
+        times.append(s.elapsed_time(e))
+    return statistics.median(times), times
+
+
+def run_report(a):
+    import numpy as np
+    import torch
+    from threadpoolctl import threadpool_limits
+
+    import oracle
+    from sequence_softmax_b200 import binding
+    from sequence_softmax_b200.inputs import WORKLOADS, sample_rows, workload_qkv
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    pk = peaks()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    threads = blas_threads()
+    for name in REPORT_WORKLOADS:
+        w = WORKLOADS[name]
+        q, k, v = workload_qkv(w, device=dev)
+        out = torch.empty_like(q)
+        lse = torch.empty(w.B, w.H, w.N, device=dev, dtype=torch.float32)
+
+        def step():
+            binding.ring_forward(q, k, v, w.n_chunks, w.causal, w.layout, out=out, lse=lse)
+
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        if binding.get_device_error() != binding.RA_OK:
+            raise RuntimeError(f"{name}: device error during warm-up")
+        n_iter = max(a.steps, 10) if w.N < (1 << 20) else max(a.steps, 3)
+        with ClockSampler(0) as clk:
+            ms, _ = _time_each(step, n_iter, flush, stream, torch)
+        if binding.get_device_error() != binding.RA_OK:
+            raise RuntimeError(f"{name}: device error in the timed region")
+        tf = w.flops() / (ms / 1e3) / 1e12
+        qn, kn, vn = (t.float().cpu().numpy() for t in (q, k, v))
+        total_pairs = w.B * w.H * w.visible_pairs()
+        with threadpool_limits(limits=threads):
+            if w.N <= 4096:
+                t0 = time.perf_counter()
+                o_ref, l_ref = oracle.attention(qn, kn, vn, w.scale, w.causal)
+                cpu_s = time.perf_counter() - t0
+                og, lg = out.float().cpu().numpy(), lse.cpu().numpy()
+                oracle_info = {"mode": "full", "cpu_s": cpu_s, "rows_per_head": w.N}
+            else:
+                rows = sample_rows(w.N, w.n_chunks, w.layout, count=a.report_rows)
+                t0 = time.perf_counter()
+                o_ref, l_ref = oracle.attention(qn, kn, vn, w.scale, w.causal, rows=rows)
+                cpu_s = time.perf_counter() - t0
+                ridx = torch.as_tensor(rows, device=dev)
+                og, lg = out[:, :, ridx].float().cpu().numpy(), lse[:, :, ridx].cpu().numpy()
+                sampled = w.B * w.H * int(((rows + 1) if w.causal else np.full(len(rows), w.N)).sum())
+                oracle_info = {"mode": "sampled rows, time extrapolated by visible pairs", "cpu_s_sampled": cpu_s,
+                               "rows_per_head": int(len(rows)), "cpu_s": cpu_s * total_pairs / sampled}
+        oracle_info.update(cores=threads, kind="fp64 NumPy oracle")
+        err = np.abs(og - o_ref)
+        fin = np.isfinite(l_ref)
+        lerr = float(np.abs(lg[fin] - l_ref[fin]).max()) if fin.any() else 0.0
+        line = {"report": name, "config": workload_config(w), "dtype": w.dtype, "ms": ms, "iters": n_iter,
+                "TFLOP/s": tf, "frac_of_burst": tf / pk["bf16_tflops"],
+                "frac_of_sustained": tf / pk.get("bf16_tflops_sustained", pk["bf16_tflops"]),
+                "peak_source": pk["source"], "l2": "flushed before every timed iteration",
+                "clocks": clk.summary(), "max_abs_err": float(err.max()), "mean_abs_err": float(err.mean()),
+                "lse_max_abs_err": lerr, "oracle": oracle_info,
+                "gpu_over_oracle": oracle_info["cpu_s"] / (ms / 1e3)}
+        print(json.dumps(line), flush=True)
+        del q, k, v, out, lse
+        torch.cuda.empty_cache()
+
+    for n, rows, d in REPORT_MERGES:
+        g = torch.Generator(device=dev).manual_seed(100 + n)
+        o_parts = torch.randn(n, rows, d, device=dev, generator=g)
+        # lse ~ N(ln Lk, 1) for KV chunks of Lk = 8192 keys, 1% of the entries -inf (chunks
+        # wholly in a row's future)
+        lse_parts = torch.randn(n, rows, device=dev, generator=g) + float(np.log(8192.0))
+        lse_parts[torch.rand(n, rows, device=dev, generator=g) < 0.01] = float("-inf")
+        out = torch.empty(rows, d, device=dev, dtype=torch.bfloat16)
+        lse = torch.empty(rows, device=dev, dtype=torch.float32)
+
+        def mstep():
+            binding.merge(o_parts, lse_parts, out=out, lse=lse)
+
+        for _ in range(3):
+            mstep()
+        torch.cuda.synchronize()
+        with ClockSampler(0) as clk:
+            ms, _ = _time_each(mstep, max(a.steps, 10), flush, stream, torch)
+        nbytes = n * rows * (4 * d + 4) + rows * (2 * d + 4)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        sr = torch.randint(0, rows, (4096,), generator=torch.Generator().manual_seed(7)).unique()
+        sri = sr.to(dev)
+        op, lp = o_parts[:, sri].cpu().numpy(), lse_parts[:, sri].cpu().numpy()
+        with threadpool_limits(limits=threads):
+            t0 = time.perf_counter()
+            o_ref, l_ref = oracle.merge(op, lp)
+            cpu_s = (time.perf_counter() - t0) * rows / len(sr)
+        err = np.abs(out[sri].float().cpu().numpy() - o_ref)
+        fin = np.isfinite(l_ref)
+        line = {"report": f"merge-n{n}-rows{rows}-d{d}", "ms": ms, "GB/s": gbs, "bytes": nbytes,
+                "frac_of_hbm": gbs / pk["hbm_gbs"], "peak_source": pk["source"],
+                "l2": "flushed before every timed iteration", "clocks": clk.summary(),
+                "max_abs_err": float(err.max()), "mean_abs_err": float(err.mean()),
+                "lse_max_abs_err": float(np.abs(lse[sri].cpu().numpy()[fin] - l_ref[fin]).max()),
+                "oracle": {"mode": f"{len(sr)} sampled rows, time extrapolated by rows", "cpu_s": cpu_s,
+                           "cores": threads, "kind": "fp64 NumPy oracle"},
+                "gpu_over_oracle": cpu_s / (ms / 1e3)}
+        print(json.dumps(line), flush=True)
+        del o_parts, lse_parts, out, lse
+        torch.cuda.empty_cache()
 
 
 if __name__ == "__main__":
