@@ -3,8 +3,11 @@
 World size 1 runs in one process. World size 2 runs two processes that share cuda:0: each
 maps the other's K||V (and, in the backward, dK||dV accumulator) buffers through CUDA IPC,
 and the library's kernels read and accumulate through those mappings; gloo carries the
-handles and the barriers between steps. The kernels of the two processes never wait on one
-another. Each rank's O, lse, dQ, dK and dV are compared with the fp64 oracle and must equal
+handles and the barriers between steps. Both ways of reading K||V run: "direct" (the
+kernels read the owner's buffer through the mapping) and "copy" (each step's block is
+pulled into a local double buffer one step ahead with one DMA copy on a copy stream, the
+copy ordered after the kernels that last read that buffer). The kernels of the two
+processes never wait on one another. Each rank's O, lse, dQ, dK and dV are compared with the fp64 oracle and must equal
 ``ring_dist``'s bit for bit (same kernels, same values, same order).
 """
 
@@ -26,7 +29,7 @@ def _local_tokens(layout, W, r):
     return np.concatenate([t0 + st * np.arange(n) for t0, st, n in ring_dist.position_segments(layout, N, W, r)])
 
 
-def _worker(rank, world, port, layout, causal, out):
+def _worker(rank, world, port, layout, causal, mode, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     import datetime
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
@@ -38,8 +41,8 @@ def _worker(rank, world, port, layout, causal, out):
         do = make_qkv(B, H, N, D, torch.bfloat16, seed=12, device="cuda")[0]
         idx = torch.as_tensor(_local_tokens(layout, world, rank), device="cuda")
         lq, lk, lv, ldo = (t[:, :, idx].contiguous() for t in (q, k, v, do))
-        o, lse = peer_ring.ring_forward_peer(lq, lk, lv, N, layout, causal)
-        grads = peer_ring.ring_backward_peer(lq, lk, lv, o, ldo, lse, N, layout, causal)
+        o, lse = peer_ring.ring_forward_peer(lq, lk, lv, N, layout, causal, mode=mode)
+        grads = peer_ring.ring_backward_peer(lq, lk, lv, o, ldo, lse, N, layout, causal, mode=mode)
         o_d, lse_d = ring_dist.ring_forward_dist(lq, lk, lv, N, layout, causal)
         grads_d = ring_dist.ring_backward_dist(lq, lk, lv, o, ldo, lse, N, layout, causal)
         torch.cuda.synchronize()
@@ -49,7 +52,7 @@ def _worker(rank, world, port, layout, causal, out):
         dist.destroy_process_group()
 
 
-def _run(world, layout, causal):
+def _run(world, layout, causal, mode="copy"):
     import oracle
     from sequence_softmax_b200.inputs import make_qkv
 
@@ -57,7 +60,7 @@ def _run(world, layout, causal):
 
     out = mp.get_context("spawn").Manager().dict()
     port = 29900 + world * 10 + os.getpid() % 500
-    mp.spawn(_worker, args=(world, port, layout, causal, out), nprocs=world, join=True)
+    mp.spawn(_worker, args=(world, port, layout, causal, mode, out), nprocs=world, join=True)
     q, k, v = make_qkv(B, H, N, D, torch.bfloat16, seed=11, device="cuda")
     do = make_qkv(B, H, N, D, torch.bfloat16, seed=12, device="cuda")[0]
     qn, kn, vn, don = (t.float().cpu().numpy() for t in (q, k, v, do))
@@ -67,7 +70,7 @@ def _run(world, layout, causal):
     for r in range(world):
         o, lse, grads, idx, same = out[r]
         idx = idx.numpy()
-        assert same, f"rank {r}: peer ring differs from ring_dist"
+        assert same, f"rank {r}: peer ring ({mode}) differs from ring_dist"
         compare(o.numpy(), lse.numpy(), o_ref[:, :, idx], l_ref[:, :, idx], "bf16", f"rank {r} {layout}")
         for full, g in zip(got, grads):
             full[:, :, idx] = g.numpy()
@@ -79,7 +82,8 @@ def test_peer_ring_world1(cuda, layout, causal):
     _run(1, layout, causal)
 
 
+@pytest.mark.parametrize("mode", ["copy", "direct"])
 @pytest.mark.parametrize("layout,causal", [("zigzag", True), ("striped", True), ("contiguous", True),
                                            ("contiguous", False)])
-def test_peer_ring_world2_shared_gpu(cuda, layout, causal):
-    _run(2, layout, causal)
+def test_peer_ring_world2_shared_gpu(cuda, layout, causal, mode):
+    _run(2, layout, causal, mode)
