@@ -63,17 +63,18 @@ struct TcCfg {
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(TC_BM, D, true);
 };
 
-// Query block owned by the CTA with index `unit` within its head, heaviest (latest tokens) first.
+// Query block of `block_rows` rows with index `unit` within its head, heaviest (latest
+// tokens) first.
 struct QBlock {
   int p;      // virtual position
   Seg seg;    // the position's segment that holds the block
   int64_t i0; // local row of tile 0 inside the segment
 };
 
-__device__ __forceinline__ QBlock decode_unit(const Plan& pl, int unit) {
+__device__ __forceinline__ QBlock decode_unit(const Plan& pl, int unit, int block_rows = 2 * TC_BM) {
   QBlock b;
   const int P = pl.P;
-  const int64_t nb = (pl.q_seg_len + 2 * TC_BM - 1) / (2 * TC_BM);
+  const int64_t nb = (pl.q_seg_len + block_rows - 1) / block_rows;
   int si = 0;
   int64_t qb;
   if (pl.layout == RA_LAYOUT_STRIPED) {
@@ -88,7 +89,7 @@ __device__ __forceinline__ QBlock decode_unit(const Plan& pl, int unit) {
     qb = nb - 1 - unit % nb;
   }
   b.seg = segment_of(pl.layout, P, pl.q_seg_len, b.p, si);
-  b.i0 = qb * (2 * TC_BM);
+  b.i0 = qb * block_rows;
   return b;
 }
 
@@ -96,82 +97,70 @@ __device__ __forceinline__ int64_t q_token(const Plan& pl, const Seg& s, int64_t
   return pl.q_tok0 + pl.q_tok_stride * (s.row0 + s.stride * i);
 }
 
-// exp2 on the FMA pipe for a share of the scores, so that the MUFU (16 results per SM
-// per clock) and the FMA pipes share the softmax's exponentials. Cody-Waite reduction
-// 2^x = 2^round(x) * 2^f, f in [-1/2, 1/2], with the degree-3 minimax polynomial printed by
-// csrc/exp2_poly.py (Remez exchange; max relative error 7.5e-5, far below bf16's 2^-9).
-// round(x) comes from adding and subtracting 1.5 * 2^23; 2^n is added into the exponent
-// field. x is clamped to >= -126 so that the exponent never wraps; 2^-126 is below any
-// visible contribution (the row max contributes >= 1).
-constexpr float EXP2_C0 = 9.999280735e-01f, EXP2_C1 = 6.932609855e-01f, EXP2_C2 = 2.426111222e-01f,
-                EXP2_C3 = 5.517166906e-02f;
-constexpr float ROUND_MAGIC = 12582912.0f;  // 1.5 * 2^23
-// Pairs of scores per group of 8 pairs that take the FMA-pipe exp2 (the rest use MUFU).
-#ifndef RA_EMU_PAIRS_OF_8
-#define RA_EMU_PAIRS_OF_8 0
-#endif
-
-__device__ __forceinline__ void exp2_poly_pair(uint64_t x2, float& p0, float& p1) {
-  float x0, x1;
-  f2_unpack(x2, x0, x1);
-  x2 = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
-  const uint64_t t2 = f2_add(x2, f2_pack(ROUND_MAGIC, ROUND_MAGIC));
-  const uint64_t n2 = f2_add(t2, f2_pack(-ROUND_MAGIC, -ROUND_MAGIC));
-  const uint64_t f2 = f2_fma(n2, f2_pack(-1.f, -1.f), x2);
-  uint64_t q2 = f2_fma(f2_pack(EXP2_C3, EXP2_C3), f2, f2_pack(EXP2_C2, EXP2_C2));
-  q2 = f2_fma(q2, f2, f2_pack(EXP2_C1, EXP2_C1));
-  q2 = f2_fma(q2, f2, f2_pack(EXP2_C0, EXP2_C0));
-  float q0, q1, t0, t1;
-  f2_unpack(q2, q0, q1);
-  f2_unpack(t2, t0, t1);
-  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+// P = exp2(s * sl2 - shift) for the 64 scores of keys 64h .. 64h + 63 of one row: P as 32
+// bf16 pairs in pk, and the sums of the even and odd pairs added into sum2a / sum2b. The
+// exponentials run on the MUFU (ex2.approx); the scale and shift are one paired FMA.
+__device__ __forceinline__ void exp_half(const uint32_t (&sr)[TC_BN], int h, uint64_t sl2x2, uint64_t negm2,
+                                         uint32_t (&pk)[32], uint64_t& sum2a, uint64_t& sum2b) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const uint64_t x2 =
+        f2_fma(f2_pack(__uint_as_float(sr[h * 64 + 2 * j]), __uint_as_float(sr[h * 64 + 2 * j + 1])), sl2x2, negm2);
+    float x0, x1;
+    f2_unpack(x2, x0, x1);
+    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+    if (j & 1) sum2b = f2_add(sum2b, f2_pack(p0, p1));
+    else sum2a = f2_add(sum2a, f2_pack(p0, p1));
+    pk[j] = pack_bf16x2(p0, p1);
+  }
 }
 
-// P = exp2(s * sl2 - shift) for one row of 128 scores: writes P as bf16 pairs into TMEM
-// columns [0, 64) at tS, arrives on bar_first_half once the first 32 columns (keys 0-63)
-// are stored, and returns the row sums of the even and odd columns. With EMU,
-// RA_EMU_PAIRS_OF_8 pairs in eight go through exp2_poly_pair (only on tiles without
-// masked scores).
-template <bool EMU>
-__device__ __forceinline__ void exp_tile(const uint32_t (&sr)[TC_BN], float sl2, float shift, uint32_t tS,
-                                         uint32_t bar_first_half, float& sum0, float& sum1) {
-  const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-shift, -shift);
-  uint64_t sum2a = f2_pack(0.f, 0.f), sum2b = sum2a;
+// Maximum of one row's 128 raw scores: eight independent chains of three-input max.
+__device__ __forceinline__ float row_max(const uint32_t (&sr)[TC_BN]) {
+#define SV(j) __uint_as_float(sr[(j)])
+  float mxc[8];
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    uint32_t pk[32];
+  for (int c = 0; c < 8; ++c) mxc[c] = fmax3(SV(2 * c), SV(2 * c + 1), SV(16 + 2 * c));
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[half * 64 + 2 * j]),
-                                         __uint_as_float(sr[half * 64 + 2 * j + 1])), sl2x2, negm2);
-      float p0, p1;
-      if (EMU && (j & 7) >= 8 - RA_EMU_PAIRS_OF_8) {
-        exp2_poly_pair(x2, p0, p1);
-      } else {
-        float x0, x1;
-        f2_unpack(x2, x0, x1);
-        p0 = ex2_approx(x0);
-        p1 = ex2_approx(x1);
-      }
-      if (j & 1) sum2b = f2_add(sum2b, f2_pack(p0, p1));
-      else sum2a = f2_add(sum2a, f2_pack(p0, p1));
-      pk[j] = pack_bf16x2(p0, p1);
-    }
-    RA_TMEM_ST32(tS + half * 32, pk);
-    if (half == 0) {
-      // P of keys 0-63 is complete: the MMA warp may start PV on it while the second
-      // half is computed.
-      tmem_wait_st();
-      tc_fence_before_sync();
-      mbar_arrive(bar_first_half);
-    }
+  for (int j = 32; j < TC_BN; j += 16) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) mxc[c] = fmax3(mxc[c], SV(j + 2 * c), SV(j + 2 * c + 1));
   }
-  float sa0, sa1, sb0, sb1;
-  f2_unpack(sum2a, sa0, sa1);
-  f2_unpack(sum2b, sb0, sb1);
-  sum0 = sa0 + sb0;
-  sum1 = sa1 + sb1;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) mxc[c] = fmaxf(mxc[c], SV(17 + 2 * c));
+#undef SV
+  return fmaxf(fmax3(mxc[0], mxc[1], mxc[2]), fmax3(mxc[3], mxc[4], fmax3(mxc[5], mxc[6], mxc[7])));
+}
+
+// O_t *= corr for this thread's row (D columns of fp32 in TMEM), 32 columns at a time.
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t tO, float corr) {
+#pragma unroll
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t orr[32];
+    RA_TMEM_LD32(tO + cc * 32, orr);
+    tmem_wait_ld();
+    RA_REG_FENCE32(orr);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * corr);
+    RA_TMEM_ST32(tO + cc * 32, orr);
+  }
+}
+
+
+// Index (0..127) of the last key of KV tile jt of segment (c, sk) that query token tq may
+// see: the segment's end and, when causal, the query's own token bound it; -1 if none.
+__device__ __forceinline__ int last_visible_key(const Plan& pl, int c, int sk, int jt, int64_t tq) {
+  const Seg ks = segment_of(pl.layout, pl.P, pl.k_seg_len, c, sk);
+  const int64_t j0 = (int64_t)jt * TC_BN;
+  int lim = (int)min((int64_t)TC_BN, ks.count - j0) - 1;
+  if (pl.causal) {
+    const int64_t tks = pl.k_tok_stride * ks.stride;
+    const int64_t tk0 = pl.k_tok0 + pl.k_tok_stride * (ks.row0 + ks.stride * j0);
+    const int64_t jl = tq < tk0 ? -1 : (tq - tk0) / tks;
+    if (jl < lim) lim = (int)jl;
+  }
+  return lim;
 }
 
 template <int D>
@@ -432,22 +421,29 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       int c = qb.p - s;
       if (c < 0) c += pl.P;
       for (int sk = 0; sk < nks && ok; ++sk) {
-        const Seg ks = segment_of(pl.layout, pl.P, pl.k_seg_len, c, sk);
-        const int ntiles = (int)((visible_prefix(pl, ks, tq_max) + TC_BN - 1) / TC_BN);
-        const int64_t tks = pl.k_tok_stride * ks.stride;
-        for (int jt = 0; jt < ntiles; ++jt, ++n) {
-          const int64_t j0 = (int64_t)jt * TC_BN;
-          const int vcount = (int)min((int64_t)TC_BN, ks.count - j0);
-          const int64_t tk0 = pl.k_tok0 + pl.k_tok_stride * (ks.row0 + ks.stride * j0);
-          const bool full = vcount == TC_BN && (!pl.causal || tk0 + tks * (TC_BN - 1) <= tq_tile_min);
-          int lim = vcount - 1;  // last visible key of this tile for this row
+        int ntiles, nfull;
+        {
+          const Seg ks = segment_of(pl.layout, pl.P, pl.k_seg_len, c, sk);
+          ntiles = (int)((visible_prefix(pl, ks, tq_max) + TC_BN - 1) / TC_BN);
+          // Leading tiles with all 128 keys present and (causal) visible to every row of the
+          // query tile: key token of the tile's last key <= the tile's first query token.
+          int64_t nf = ks.count / TC_BN;
           if (pl.causal) {
-            const int64_t jl = tq < tk0 ? -1 : (tq - tk0) / tks;
-            if (jl < lim) lim = (int)jl;
+            const int64_t tks = pl.k_tok_stride * ks.stride;
+            const int64_t t0 = pl.k_tok0 + pl.k_tok_stride * ks.row0;
+            const int64_t slack = tq_tile_min - t0 - tks * (TC_BN - 1);
+            const int64_t vis = slack < 0 ? 0 : slack / (tks * TC_BN) + 1;
+            if (vis < nf) nf = vis;
           }
+          nfull = (int)min(nf, (int64_t)ntiles);
+        }
+        for (int jt = 0; jt < ntiles; ++jt, ++n) {
+          const bool full = jt < nfull;
           if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(t), (uint32_t)n & 1u, abort_flag))) { ok = false; break; }
           tc_fence_after_sync();
           uint32_t sr[TC_BN];
+          // S_t of this row from tensor memory; keys after this row's last visible one are
+          // masked on a tile that straddles the causal diagonal or the segment's end.
           RA_TMEM_LD32(tS + 0, (sr + 0));
           RA_TMEM_LD32(tS + 32, (sr + 32));
           RA_TMEM_LD32(tS + 64, (sr + 64));
@@ -458,52 +454,48 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           RA_REG_FENCE32((sr + 64));
           RA_REG_FENCE32((sr + 96));
           if (!full) {
+            const int lim = last_visible_key(pl, c, sk, jt, tq);
 #pragma unroll
             for (int j = 0; j < TC_BN; ++j) sr[j] = (j <= lim) ? sr[j] : __float_as_uint(-INFINITY);
           }
-#define SV(j) __uint_as_float(sr[(j)])
-          float mxc[8];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) mxc[c] = fmax3(SV(2 * c), SV(2 * c + 1), SV(16 + 2 * c));
-#pragma unroll
-          for (int j = 32; j < TC_BN; j += 16) {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) mxc[c] = fmax3(mxc[c], SV(j + 2 * c), SV(j + 2 * c + 1));
-          }
-#pragma unroll
-          for (int c = 0; c < 8; ++c) mxc[c] = fmaxf(mxc[c], SV(17 + 2 * c));
-          const float mx = fmaxf(fmax3(mxc[0], mxc[1], mxc[2]), fmax3(mxc[3], mxc[4], fmax3(mxc[5], mxc[6], mxc[7]))) * sl2;
-          // Running max update (conditional rescale, see the file comment).
-          float corr = 1.f;
-          bool rescale = false;
-          if (m == -INFINITY) {
-            m = mx;  // first visible keys of this row: O and l are still 0
-          } else if (mx > m + RESCALE_LOG2) {
-            corr = ex2_approx(m - mx);
-            m = mx;
-            l *= corr;
-            rescale = true;
-          }
-          if (__any_sync(0xffffffffu, rescale) && n > 0) {
-#pragma unroll
-            for (int cc = 0; cc < D / 32; ++cc) {
-              uint32_t orr[32];
-              RA_TMEM_LD32(tO + cc * 32, orr);
-              tmem_wait_ld();
-              RA_REG_FENCE32(orr);
-#pragma unroll
-              for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * corr);
-              RA_TMEM_ST32(tO + cc * 32, orr);
+          const uint64_t sl2x2 = f2_pack(sl2, sl2);
+          uint64_t sum2a = f2_pack(0.f, 0.f), sum2b = sum2a;
+          uint32_t pk[32];
+          // Running max update (conditional rescale, see the file comment): m moves only
+          // when the tile's max exceeds it by more than RESCALE_LOG2; O and l are then
+          // scaled by corr.
+          auto update_max = [&](float mx) {
+            float corr = 1.f;
+            bool rescale = false;
+            if (m == -INFINITY) {
+              m = mx;  // first visible keys of this row: O and l are still 0
+            } else if (mx > m + RESCALE_LOG2) {
+              corr = ex2_approx(m - mx);
+              m = mx;
+              l *= corr;
+              rescale = true;
             }
+            if (__any_sync(0xffffffffu, rescale) && n > 0) rescale_o<D>(tO, corr);
+          };
+          // The online update as the pages state it: the tile's row max first, then the
+          // exponentials with the (conditionally) updated running max.
+          update_max(row_max(sr) * sl2);
+          exp_half(sr, 0, sl2x2, f2_pack(m == -INFINITY ? 0.f : -m, m == -INFINITY ? 0.f : -m), pk, sum2a, sum2b);
+          // P of keys 0-63 is complete: the MMA warp may start PV on it while the second half
+          // is computed.
+          RA_TMEM_ST32(tS, pk);
+          tmem_wait_st();
+          tc_fence_before_sync();
+          mbar_arrive(bar_p_half(t));
+          {
+            const float shift = m == -INFINITY ? 0.f : m;
+            exp_half(sr, 1, sl2x2, f2_pack(-shift, -shift), pk, sum2a, sum2b);
           }
-          const float shift = (m == -INFINITY) ? 0.f : m;
-          float sum0, sum1;
-          if (full)
-            exp_tile<true>(sr, sl2, shift, tS, bar_p_half(t), sum0, sum1);
-          else
-            exp_tile<false>(sr, sl2, shift, tS, bar_p_half(t), sum0, sum1);
-#undef SV
-          l += sum0 + sum1;
+          RA_TMEM_ST32(tS + 32, pk);
+          float sa0, sa1, sb0, sb1;
+          f2_unpack(sum2a, sa0, sa1);
+          f2_unpack(sum2b, sb0, sb1);
+          l += (sa0 + sb0) + (sa1 + sb1);
           tmem_wait_st();
           tc_fence_before_sync();
           mbar_arrive(bar_p_full(t));

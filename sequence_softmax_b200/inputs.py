@@ -79,6 +79,13 @@ WORKLOADS = {
         Workload("seq128k-d128-causal-striped16", 1, 32, 131072, 128, "bf16", True, 16, "striped", 4),
         Workload("seq1m-d128-causal-zigzag16", 1, 8, 1048576, 128, "bf16", True, 16, "zigzag", 5,
                  notes="1M-token causal zig-zag forward emitting O and per-row lse"),
+        # Head subsets of the two benchmark workloads for profiler counter captures (about
+        # 1 GB on the device): the kernels walk the heads one after another (head-major CTA
+        # order), so per-head traffic and time match the full workloads'.
+        Workload("seq1m-d128-causal-zigzag16-h1", 1, 1, 1048576, 128, "bf16", True, 16, "zigzag", 5,
+                 notes="one head of the 1M-token workload (counter captures)"),
+        Workload("seq128k-d128-causal-zigzag16-h4", 1, 4, 131072, 128, "bf16", True, 16, "zigzag", 4,
+                 notes="four heads of the 128K-token zig-zag workload (backward counter captures)"),
     ]
 }
 
