@@ -1,29 +1,31 @@
-"""Ring attention across GPUs with every K/V block read in place from its owner's memory
+"""Ring attention across GPUs with every K/V block read from its owner's memory
 (``ring_forward_peer``, ``ring_backward_peer``).
 
 ``ring_dist`` moves K||V to the successor at every step with the process group's
 point-to-point calls. GPUs joined by NVLink / NVSwitch can address each other's memory, so
 here no message is sent: each rank maps the other ranks' K||V buffers once (CUDA IPC
-handles, exchanged through the process group) and at step s hands the library the owner's
-pointers for block (rank - s) mod W. The kernels' TMA loads then fetch the tiles from the
-owner's memory as they consume them: the transfer overlaps the compute tile by tile inside
-the kernel, and no copy of a remote block is ever made. Visiting order, causal skip and the
-online-softmax merge are those of ``ring_dist`` ("Ring Attention 논문 분석", listing
-``ring_attention_forward``; gpumode lecture 013 notes, log-sum-exp merge), with the same
-kernels on the same values in the same order, so the two give bit-identical results.
+handles, exchanged through the process group) and at step s reads block (rank - s) mod W
+from its owner. Visiting order, causal skip and the online-softmax merge are those of
+``ring_dist`` ("Ring Attention 논문 분석", listing ``ring_attention_forward``; gpumode
+lecture 013 notes, log-sum-exp merge), with the same kernels on the same values in the same
+order, so the two give bit-identical results.
+
+How K||V is read (``mode``): "copy" (the default) pulls each step's block one step ahead
+into a local double buffer with one DMA copy (``cudaMemcpyAsync`` on a copy stream), so the
+block crosses NVLink once while the previous step computes, and the kernels' re-reads of
+its tiles (every query tile pair streams the whole block) stay in this GPU's L2 and memory:
+the survey's "receive into local HBM, then local TMA". "direct" hands the kernels the
+owner's pointers, so their TMA loads fetch every tile over NVLink as the MMA pipeline
+consumes it, re-reads included.
 
 Backward: block c's fp32 dK and dV accumulators live in c's owner's memory. At step s the
 rank holding block (rank - s) mod W adds its queries' contributions into them in place
 (``ra_partial_backward`` stores through the mapped pointers) and into its own dQ. Block c
-is written by rank c + s at step s, so a barrier between steps leaves exactly one writer
-per block at a time, and when the last step ends each owner holds its blocks' dK and dV:
-the listing ``ring_attention_backward``'s reduce, read as that sum, with no return hop.
-
-How K||V is read (``mode``): "direct" hands the kernels the owner's pointers, as above;
-"copy" pulls each step's block one step ahead into a local double buffer with one DMA copy
-(``cudaMemcpyAsync`` on a copy stream), so the block crosses NVLink once while the previous
-step computes and the kernels' re-reads of its tiles (every query tile pair streams the
-whole block) stay in this GPU's L2 and memory instead of crossing NVLink again.
+is written by rank c + s at step s; each writer's stream waits, through an interprocess
+CUDA event, for the previous writer's kernels (``_StepOrder``), so there is one writer per
+block at a time without any host waiting for GPU work, and when the last step ends each
+owner holds its blocks' dK and dV: the listing ``ring_attention_backward``'s reduce, read
+as that sum, with no return hop.
 
 Only the library's kernels and the DMA copies touch another rank's memory (plain per-CTA
 TMA loads, the backward's accumulator stores, ``cudaMemcpyAsync``); merges, casts
@@ -156,6 +158,58 @@ def _fence(group, device_work: bool):
     dist.barrier(group)
 
 
+# _StepOrder instances created so far per group (by its global ranks): every member makes
+# them in the same order, so the count names an instance consistently across processes.
+_ORDER_SEQ: dict = {}
+
+
+class _StepOrder:
+    """Device-side order between consecutive writers of a block's dK/dV accumulators.
+
+    At step s rank r adds into the accumulators of block (r - s) mod W, which rank r - 1
+    wrote at step s - 1. After enqueueing step s, every rank records its interprocess CUDA
+    event for step s on its stream and publishes that in the process group's store; before
+    step s + 1, its successor waits (on the host) for that key only, then makes its stream
+    wait on the event (cudaStreamWaitEvent). No host waits for GPU work, so the steps'
+    kernels queue back to back, and each event is recorded once per call, so a wait always
+    refers to the intended step. Without CUDA (host tensors) the key alone orders the steps.
+    """
+
+    def __init__(self, group, device: torch.device | None):
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        self.cuda = device is not None
+        if self.world == 1:
+            return
+        ranks = tuple(dist.get_process_group_ranks(group) if group is not None else range(self.world))
+        seq = _ORDER_SEQ.get(ranks, 0)
+        _ORDER_SEQ[ranks] = seq + 1
+        self.prefix = f"ra_peer_ring_order/{'-'.join(map(str, ranks))}/{seq}"
+        self.store = dist.distributed_c10d._get_default_store()
+        if self.cuda:
+            self.mine = [torch.cuda.Event(interprocess=True) for _ in range(self.world)]
+            handles = [None] * self.world
+            dist.all_gather_object(handles, [e.ipc_handle() for e in self.mine], group=group)
+            prev = (self.rank - 1) % self.world
+            self.pred = [torch.cuda.Event.from_ipc_handle(device, h) for h in handles[prev]]
+
+    def after_step(self, s: int):
+        """Step s's kernels are enqueued: publish their completion to the successor."""
+        if self.world == 1:
+            return
+        if self.cuda:
+            self.mine[s].record(torch.cuda.current_stream())
+        self.store.set(f"{self.prefix}/{self.rank}/{s}", "1")
+
+    def before_step(self, s: int):
+        """Step s may write what the predecessor wrote at step s - 1: wait for it."""
+        if s == 0 or self.world == 1:
+            return
+        self.store.wait([f"{self.prefix}/{(self.rank - 1) % self.world}/{s - 1}"])
+        if self.cuda:
+            torch.cuda.current_stream().wait_event(self.pred[s - 1])
+
+
 class _Blocks:
     """The K||V block of each ring step, as the tensor this rank's kernels read.
 
@@ -219,7 +273,7 @@ def _check_local(q_local, others, segs):
 
 
 def ring_forward_peer(q_local, k_local, v_local, N: int, layout: str = "contiguous", causal: bool = False,
-                      scale: float | None = None, group=None, kernels=None, share=None, mode: str = "direct"):
+                      scale: float | None = None, group=None, kernels=None, share=None, mode: str = "copy"):
     """Exact attention over N tokens split across the ranks of `group`, reading each K/V
     block from its owner's memory.
 
@@ -227,8 +281,8 @@ def ring_forward_peer(q_local, k_local, v_local, N: int, layout: str = "contiguo
     [B, H, N/W, d] on this rank's GPU hold the tokens of virtual position `rank` in
     increasing token order; returns (O_local in the input dtype, lse_local fp32).
     ``kernels`` (default: the library binding) provides ``partial`` and ``merge``. ``mode``:
-    "direct" (the kernels read the owner's buffer) or "copy" (each block pulled into a local
-    buffer one step ahead; see ``_Blocks``).
+    "copy" (the default: each block pulled into a local buffer one step ahead, so it crosses
+    NVLink once; see ``_Blocks``) or "direct" (the kernels read the owner's buffer).
     """
     kern = binding if kernels is None else kernels
     share = PeerBuffers if share is None else share
@@ -276,7 +330,7 @@ def ring_forward_peer(q_local, k_local, v_local, N: int, layout: str = "contiguo
 
 def ring_backward_peer(q_local, k_local, v_local, o_local, do_local, lse_local, N: int, layout: str = "contiguous",
                        causal: bool = False, scale: float | None = None, group=None, kernels=None, share=None,
-                       mode: str = "direct"):
+                       mode: str = "copy"):
     """Gradients (dQ, dK, dV) of ``ring_forward_peer``'s output for upstream gradient
     do_local, every block's dK and dV accumulated in place in its owner's memory.
 
@@ -312,8 +366,10 @@ def ring_backward_peer(q_local, k_local, v_local, o_local, do_local, lse_local, 
     try:
         sched = ring_schedule(rank, world)
         blocks = _Blocks(mode, peers_kv, sched, kv)
+        order = _StepOrder(group, kv.device if kv.is_cuda else None)
         _fence(group, kv.is_cuda)
         for s, src in enumerate(sched):
+            order.before_step(s)
             kv_src, acc_src = blocks.get(s), peers_acc.views[src]
             for ki, kseg in enumerate(position_segments(layout, N, world, src)):
                 for qi, qseg in enumerate(segs):
@@ -324,7 +380,8 @@ def ring_backward_peer(q_local, k_local, v_local, o_local, do_local, lse_local, 
                                           q_tok0=qseg[0], q_tok_stride=qseg[1], k_tok0=kseg[0], k_tok_stride=kseg[1])
             blocks.done(s)
             # block src's next writer (rank + 1, next step) starts after these additions
-            _fence(group, kv.is_cuda)
+            order.after_step(s)
+        _fence(group, kv.is_cuda)  # every rank's additions are complete before the owners read them
         own = peers_acc.views[rank]
         dk = torch.cat(list(own[0]), dim=2).to(k_local.dtype)
         dv = torch.cat(list(own[1]), dim=2).to(v_local.dtype)

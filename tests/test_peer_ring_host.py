@@ -112,3 +112,40 @@ def test_peer_ring_forward_and_backward(world, layout, causal, mode):
         assert np.abs(lf - lse[:, :, idx]).max() <= 1e-5
         for gg, rr in zip(got, ref):
             assert np.abs(gg - rr[:, :, idx]).max() <= 1e-4 * max(1.0, np.abs(rr).max())
+
+
+def _order_main(rank, world, port, out):
+    import random
+    import time as _time
+
+    from sequence_softmax_b200 import peer_ring
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        rnd = random.Random(rank)
+        spans = []
+        for _call in range(2):  # two calls: the second must not see the first one's keys
+            order = peer_ring._StepOrder(None, None)
+            for s in range(world):
+                order.before_step(s)
+                t0 = _time.time()
+                _time.sleep(rnd.uniform(0.0, 0.05))
+                spans.append((_call, s, t0, _time.time()))
+                order.after_step(s)
+        out[rank] = spans
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_step_order_follows_the_predecessor(world):
+    """Step s of rank r starts only after step s - 1 of rank r - 1 (the previous writer of
+    the block rank r writes at step s) has ended, in every call."""
+    out = mp.get_context("spawn").Manager().dict()
+    port = 29750 + 13 * world + os.getpid() % 300
+    mp.spawn(_order_main, args=(world, port, out), nprocs=world, join=True)
+    for r in range(world):
+        prev = {(c, s): (t0, t1) for c, s, t0, t1 in out[(r - 1) % world]}
+        for c, s, t0, _ in out[r]:
+            if s > 0:
+                assert t0 >= prev[(c, s - 1)][1]
