@@ -63,18 +63,17 @@ struct TcCfg {
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(TC_BM, D, true);
 };
 
-// Query block of `block_rows` rows with index `unit` within its head, heaviest (latest
-// tokens) first.
+// Query block owned by the CTA with index `unit` within its head, heaviest (latest tokens) first.
 struct QBlock {
   int p;      // virtual position
   Seg seg;    // the position's segment that holds the block
   int64_t i0; // local row of tile 0 inside the segment
 };
 
-__device__ __forceinline__ QBlock decode_unit(const Plan& pl, int unit, int block_rows = 2 * TC_BM) {
+__device__ __forceinline__ QBlock decode_unit(const Plan& pl, int unit) {
   QBlock b;
   const int P = pl.P;
-  const int64_t nb = (pl.q_seg_len + block_rows - 1) / block_rows;
+  const int64_t nb = (pl.q_seg_len + 2 * TC_BM - 1) / (2 * TC_BM);
   int si = 0;
   int64_t qb;
   if (pl.layout == RA_LAYOUT_STRIPED) {
@@ -89,7 +88,7 @@ __device__ __forceinline__ QBlock decode_unit(const Plan& pl, int unit, int bloc
     qb = nb - 1 - unit % nb;
   }
   b.seg = segment_of(pl.layout, P, pl.q_seg_len, b.p, si);
-  b.i0 = qb * block_rows;
+  b.i0 = qb * (2 * TC_BM);
   return b;
 }
 
@@ -161,6 +160,14 @@ __device__ __forceinline__ int last_visible_key(const Plan& pl, int c, int sk, i
     if (jl < lim) lim = (int)jl;
   }
   return lim;
+}
+
+// P ready: this thread's tcgen05.st of P are complete; every softmax thread of the tile
+// arrives (one arrival per warp measured slower).
+__device__ __forceinline__ void arrive_p_ready(uint32_t bar) {
+  tmem_wait_st();
+  tc_fence_before_sync();
+  mbar_arrive(bar);
 }
 
 template <int D>
@@ -484,9 +491,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           // P of keys 0-63 is complete: the MMA warp may start PV on it while the second half
           // is computed.
           RA_TMEM_ST32(tS, pk);
-          tmem_wait_st();
-          tc_fence_before_sync();
-          mbar_arrive(bar_p_half(t));
+          arrive_p_ready(bar_p_half(t));
           {
             const float shift = m == -INFINITY ? 0.f : m;
             exp_half(sr, 1, sl2x2, f2_pack(-shift, -shift), pk, sum2a, sum2b);
@@ -496,9 +501,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           f2_unpack(sum2a, sa0, sa1);
           f2_unpack(sum2b, sb0, sb1);
           l += (sa0 + sb0) + (sa1 + sb1);
-          tmem_wait_st();
-          tc_fence_before_sync();
-          mbar_arrive(bar_p_full(t));
+          arrive_p_ready(bar_p_full(t));
         }
       }
     }

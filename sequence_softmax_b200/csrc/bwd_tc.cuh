@@ -47,8 +47,8 @@ namespace ra {
 constexpr int BW_THREADS = 384;
 constexpr int BW_WARP_PRODUCER = 8;
 constexpr int BW_WARP_MMA = 9;
-constexpr int BW_REGS_MATH = 216;   // 2 x 216 + 72 = 504 = 168 * 384 / 128
-constexpr int BW_REGS_OTHER = 72;
+constexpr int BW_REGS_MATH = 224;   // 2 x 224 + 56 = 504 = 168 * 384 / 128 (216 / 72 spills)
+constexpr int BW_REGS_OTHER = 56;
 constexpr int BW_TMEM_COLS = 512;
 
 template <int D>

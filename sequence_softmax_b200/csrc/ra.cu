@@ -9,7 +9,6 @@
 #include "common.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
-#include "attn_tc2.cuh"
 #include "merge.cuh"
 #include "bwd.cuh"
 #include "bwd_tc.cuh"
@@ -61,14 +60,13 @@ EncodeTiledFn encode_fn() {
 }
 
 // 4-D view of a [BH, rows, d] bf16 buffer as (d, S, rows / S, BH): a box of 64 columns x
-// 1 x box_rows rows x 1 selects box_rows rows spaced S apart (S = P for the striped layout,
-// else 1).
-bool make_tile_map(CUtensorMap* map, const void* base, int BH, int64_t rows, int d, int S, int box_rows = TC_BN) {
+// 1 x 128 rows x 1 selects 128 rows spaced S apart (S = P for the striped layout, else 1).
+bool make_tile_map(CUtensorMap* map, const void* base, int BH, int64_t rows, int d, int S) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)S, (cuuint64_t)(rows / S), (cuuint64_t)BH};
   const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)S * d * 2, (cuuint64_t)rows * d * 2};
-  const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)TC_BN, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -109,57 +107,8 @@ ra_status launch_tc(const Plan& pl, int S, cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
-// The d = 128 forward on CTA pairs (attn_tc2.cuh): clusters of two CTAs, 512 query rows each.
-ra_status launch_tc2(const Plan& pl, int S, cudaStream_t stream) {
-  using C = Tc2Cfg;
-  CUtensorMap mq, mk, mv;
-  if (!make_tile_map(&mq, pl.q, pl.BH, pl.q_rows, C::D, S) ||
-      !make_tile_map(&mk, pl.k, pl.BH, pl.k_rows, C::D, S, TC_BN / 2) ||
-      !make_tile_map(&mv, pl.v, pl.BH, pl.k_rows, C::D, S))
-    return RA_ERR_CUDA;
-  static bool attr_done[64] = {};
-  static std::mutex mu;
-  {
-    std::lock_guard<std::mutex> g(mu);
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return RA_ERR_CUDA;
-    if (dev < 0 || dev >= 64) return RA_ERR_UNSUPPORTED;
-    if (!attr_done[dev]) {
-      if (cudaFuncSetAttribute(attn_fwd_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-          cudaSuccess)
-        return RA_ERR_CUDA;
-      attr_done[dev] = true;
-    }
-  }
-  const int64_t nb = (pl.q_seg_len + TC2_BLOCK_ROWS - 1) / TC2_BLOCK_ROWS;
-  const int64_t pairs = nb * (int64_t)pl.P * num_segments(pl.layout) * pl.BH;
-  if (pairs <= 0) return RA_OK;
-  if (2 * pairs > 0x7FFFFFFFll) return RA_ERR_UNSUPPORTED;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
-  cfg.blockDim = dim3(TC_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, attn_fwd_tc2_kernel, mq, mk, mv, pl) != cudaSuccess) return RA_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
-}
-
-// Built with RA_PAIR_FORWARD=1, the ring forward's bf16, d = 128 problems (O in bf16) run on
-// CTA pairs (attn_tc2.cuh).
-#ifndef RA_PAIR_FORWARD
-#define RA_PAIR_FORWARD 0
-#endif
-
 ra_status launch_attention(const Plan& pl, ra_dtype dt, int S, cudaStream_t stream) {
   if (dt == RA_BF16) {
-    if (pl.d == 128 && RA_PAIR_FORWARD && !pl.out_f32) return launch_tc2(pl, S, stream);
     if (pl.d == 128) return launch_tc<128>(pl, S, stream);
     if (pl.d == 64) return launch_tc<64>(pl, S, stream);
     return RA_ERR_UNSUPPORTED;
