@@ -12,7 +12,7 @@ N(0, 1)), resident in HBM and 6.4 GB in total, so they exceed the 126 MB L2 betw
 Rank 0 prints one JSON line. With N > 1 (torchrun), the default (--multi ring) runs the
 pages' own partition of the same workload over the N GPUs: each rank holds the tokens of one
 virtual ring position (zig-zag: chunks r and 2N-1-r), keeps its queries, and K||V rotates
-around the ring over NCCL while ra_partial + ra_merge fold each block into the running state
+around the ring over NCCL while ra_partial_fold folds each block into the running state
 ("Ring Attention 논문 분석", listing ring_attention_forward). The total work is fixed (strong
 scaling). --multi replicas instead runs an independent replica of the workload per rank
 (weak scaling, no collective on the data path). Time is the max over ranks of CUDA-event
@@ -508,7 +508,7 @@ class CountingKernels:
         fn = getattr(self._binding, name)
 
         def call(*args, **kwargs):
-            self.launches += 1  # partial, merge: one kernel launch per call
+            self.launches += 1  # partial_fold: one kernel launch per call
             return fn(*args, **kwargs)
         return call
 
@@ -581,9 +581,9 @@ def run_ring(a, w):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
         "roofline": {"bound": "tensor", "achieved": per_gpu, "peak": peak, "unit": "TFLOP/s",
                      "frac": per_gpu / peak, "traffic": None, "peak_source": f"{pk['source']} bf16 burst",
-                     "note": "per-GPU step throughput of the ring (ra_partial's attn_fwd_tc_kernel<128> "
-                             "launches plus ra_merge and the exchange), not one launch",
-                     "kernel": "attn_fwd_tc_kernel<128> via ra_partial"},
+                     "note": "per-GPU step throughput of the ring (ra_partial_fold's attn_fwd_tc_kernel<128> "
+                             "launches and the exchange), not one launch",
+                     "kernel": "attn_fwd_tc_kernel<128> via ra_partial_fold"},
         "clocks": clk.summary(),
         "gpu_launches": int(launches.item()),
     }

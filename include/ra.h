@@ -89,6 +89,27 @@ ra_status ra_partial(const void* q, const void* k, const void* v, ra_dtype dt,
                      float* o_partial, float* lse, cudaStream_t stream);
 
 /*
+ * ra_partial_fold -- ra_partial whose result is merged, in the same kernel, into a running
+ * partial state held by the caller: the per-step update of the ring ([BLOG]
+ * ring_attention_forward: the state (m, l, o) is carried from step to step and every new KV
+ * chunk is folded into it; [LECTURE] log-sum-exp passage for the merge in (O, lse) form).
+ *
+ *   q, k, v, dt, B, H, Lq, Lk, d, scale, causal, q_tok0 ... k_tok_stride: as ra_partial
+ *   o_state    [B, H, Lq, d]  fp32, read and written: the normalised state O
+ *   lse_state  [B, H, Lq]     fp32, read and written: the state's lse (-inf: nothing seen yet)
+ *
+ * Afterwards (o_state, lse_state) equal, bit for bit, what ra_partial into a scratch state
+ * followed by ra_merge (n = 2, parts [state, new], fp32 output) would leave, without the
+ * scratch state, the merge launch or the copies back. Start a ring with o_state = 0 and
+ * lse_state = -inf. Lq == 0 and Lk == 0 leave the state as it is. The state must not overlap
+ * q, k or v.
+ */
+ra_status ra_partial_fold(const void* q, const void* k, const void* v, ra_dtype dt,
+                          int B, int H, int64_t Lq, int64_t Lk, int d, float scale, int causal,
+                          int64_t q_tok0, int64_t q_tok_stride, int64_t k_tok0, int64_t k_tok_stride,
+                          float* o_state, float* lse_state, cudaStream_t stream);
+
+/*
  * ra_merge -- lse-weighted combination of n partial states, from the associativity
  * lse(x) = lse([lse(x1), lse(x2)]) ([LECTURE] log-sum-exp passage):
  *   L = max_i lse_i + log sum_i exp(lse_i - max_i lse_i),   O = sum_i exp(lse_i - L) O_i.
@@ -246,7 +267,7 @@ ra_status ra_selftest_wait_timeout(int64_t limit_ns, cudaStream_t stream);
 
 /* ABI version of this header (incremented on any signature change); ra_abi_version()
  * returns the version the library was built with, so a caller can compare the two. */
-#define RA_ABI_VERSION 2
+#define RA_ABI_VERSION 3
 int ra_abi_version(void);
 
 #ifdef __cplusplus

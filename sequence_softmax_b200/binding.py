@@ -20,13 +20,15 @@ library_path = os.environ.get("RA_LIBRARY", os.path.join(_PKG, "libra.so"))
 RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_CUDA, RA_ERR_TIMEOUT, RA_ERR_DEVICE_BOUNDS = range(6)
 RA_F32, RA_BF16 = 0, 1
 LAYOUTS = {"contiguous": 0, "striped": 1, "zigzag": 2}
-ABI_VERSION = 2  # the ABI these signatures describe (ra_abi_version() of a matching library)
+ABI_VERSION = 3  # the ABI these signatures describe (ra_abi_version() of a matching library)
 
 # name -> (restype, argtypes) of every symbol include/ra.h declares
 _i64, _i32, _f32, _vp = ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_void_p
 SIGNATURES = {
     "ra_partial": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i64, _i64, _i32, _f32, _i32,
                           _i64, _i64, _i64, _i64, _vp, _vp, _vp]),
+    "ra_partial_fold": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i64, _i64, _i32, _f32, _i32,
+                               _i64, _i64, _i64, _i64, _vp, _vp, _vp]),
     "ra_merge": (_i32, [_vp, _vp, _i32, _i64, _i32, _vp, _i32, _vp, _vp]),
     "ra_ring_forward": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i64, _i32, _f32, _i32, _i32,
                                _i32, _vp, _vp, _vp]),
@@ -137,6 +139,27 @@ def partial(q, k, v, causal: bool = False, scale: float | None = None,
                            out.data_ptr(), lse.data_ptr(), _stream_ptr(stream))
     _check(st, "ra_partial")
     return out, lse
+
+
+def partial_fold(q, k, v, o_state, lse_state, causal: bool = False, scale: float | None = None,
+                 q_tok0: int = 0, q_tok_stride: int = 1, k_tok0: int = 0, k_tok_stride: int = 1, stream=None):
+    """One query block against one KV chunk, merged in place into the running state
+    (o_state fp32 [B,H,Lq,d], lse_state fp32 [B,H,Lq]); returns them."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o_state, "o_state"), (lse_state, "lse_state")):
+        _dev(t, n)
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    if k.shape != (B, H, Lk, d) or v.shape != k.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("k and v must be [B, H, Lk, d] with q's B, H, d and dtype")
+    if o_state.shape != (B, H, Lq, d) or lse_state.shape != (B, H, Lq) or o_state.dtype != torch.float32 \
+            or lse_state.dtype != torch.float32:
+        raise ValueError("the state is o_state fp32 [B, H, Lq, d] and lse_state fp32 [B, H, Lq]")
+    scale = d ** -0.5 if scale is None else float(scale)
+    st = load().ra_partial_fold(q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q), B, H, Lq, Lk, d, scale,
+                                int(bool(causal)), q_tok0, q_tok_stride, k_tok0, k_tok_stride,
+                                o_state.data_ptr(), lse_state.data_ptr(), _stream_ptr(stream))
+    _check(st, "ra_partial_fold")
+    return o_state, lse_state
 
 
 def merge(o_parts, lse_parts, out_dtype=torch.bfloat16, with_lse: bool = True, out=None, lse=None,

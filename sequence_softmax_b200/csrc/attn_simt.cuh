@@ -96,17 +96,28 @@ attn_fwd_simt_f32_kernel(const Plan pl, int64_t rows_per_pos) {
     }
   }
   const float inv_l = l > 0.f ? 1.f / l : 0.f;
-  float* op = static_cast<float*>(pl.o) + ((int64_t)bh * pl.q_rows + qrow) * d;
+  const float lse_row = l > 0.f ? m + logf(l) : -INFINITY;
+  const int64_t orow = (int64_t)bh * pl.q_rows + qrow;
+  float* op = static_cast<float*>(pl.o) + orow * d;
+  // Folding into a running state: every lane reads the state's lse before any lane writes it.
+  FoldWeights fw{lse_row, 0.f, 1.f};
+  if (pl.fold) {
+    fw = fold_weights(pl.lse[orow], lse_row);
+    __syncwarp();
+  }
 #pragma unroll
   for (int t = 0; t < SIMT_DMAX / 32; ++t) {
     const int e = lane + 32 * t;
-    if (e < d) op[e] = acc[t] * inv_l;
+    if (e < d) {
+      const float o_new = acc[t] * inv_l;
+      op[e] = pl.fold ? fmaf(fw.w_new, o_new, fmaf(fw.w_state, op[e], 0.f)) : o_new;
+    }
   }
-  if (lane == 0 && pl.lse != nullptr)
-    pl.lse[(int64_t)bh * pl.q_rows + qrow] = l > 0.f ? m + logf(l) : -INFINITY;
+  if (lane == 0 && pl.lse != nullptr) pl.lse[orow] = fw.L;
 }
 
-// Writes the empty state (O = 0, lse = -inf) for every row: ra_partial with Lk == 0.
+// Writes the empty state (O = 0, lse = -inf) for every row: ra_partial with Lk == 0 (the
+// folding variant leaves the running state as it is instead).
 __global__ void fill_empty_kernel(float* o, float* lse, int64_t rows, int d) {
   const int64_t n = rows * d;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {

@@ -512,6 +512,12 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const int64_t mrow = qb.seg.row0 + qb.seg.stride * li;
       const int64_t orow = (int64_t)bh * pl.q_rows + mrow;
       const bool row_ok = row_valid && in_bounds(mrow < pl.q_rows);
+      const float lse_row = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      // Folding into a caller's running state (fp32 output only): this row's weights, with
+      // the merge kernel's arithmetic; the thread owns the row, so it reads the state before
+      // writing it.
+      FoldWeights fw{lse_row, 0.f, 1.f};
+      if (pl.fold && row_ok) fw = fold_weights(pl.lse[orow], lse_row);
       if (T > 0) tc_fence_after_sync();
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
@@ -528,9 +534,18 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           if (pl.out_f32) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(pl.o) + orow * D + cc * 32);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              dst[j] = make_float4(__uint_as_float(orr[4 * j]) * inv_l, __uint_as_float(orr[4 * j + 1]) * inv_l,
-                                   __uint_as_float(orr[4 * j + 2]) * inv_l, __uint_as_float(orr[4 * j + 3]) * inv_l);
+            for (int j = 0; j < 8; ++j) {
+              float4 o = make_float4(__uint_as_float(orr[4 * j]) * inv_l, __uint_as_float(orr[4 * j + 1]) * inv_l,
+                                     __uint_as_float(orr[4 * j + 2]) * inv_l, __uint_as_float(orr[4 * j + 3]) * inv_l);
+              if (pl.fold) {
+                const float4 st = dst[j];
+                o.x = fmaf(fw.w_new, o.x, fmaf(fw.w_state, st.x, 0.f));
+                o.y = fmaf(fw.w_new, o.y, fmaf(fw.w_state, st.y, 0.f));
+                o.z = fmaf(fw.w_new, o.z, fmaf(fw.w_state, st.z, 0.f));
+                o.w = fmaf(fw.w_new, o.w, fmaf(fw.w_state, st.w, 0.f));
+              }
+              dst[j] = o;
+            }
           } else {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(pl.o) + orow * D + cc * 32);
 #pragma unroll
@@ -545,8 +560,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           }
         }
       }
-      if (row_ok && pl.lse != nullptr)
-        pl.lse[orow] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      if (row_ok && pl.lse != nullptr) pl.lse[orow] = fw.L;
     }
   }
 

@@ -68,6 +68,7 @@ struct Plan {
   int layout;        // ra_layout
   int causal;
   int out_f32;       // 1: O written as fp32 (partial states); 0: O in the input dtype
+  int fold;          // 1: o / lse hold a running state that the result is merged into
   int64_t q_rows;    // rows per head in the Q / O buffers
   int64_t k_rows;    // rows per head in the K / V buffers
   int64_t q_seg_len; // rows per Q segment
@@ -370,6 +371,29 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Merging a running partial state (lse_state) with a new one (lse_new): L and the two
+// weights, with exactly the operations merge_kernel performs for the parts [state, new]
+// (max, shift, sum of expf, logf, expf), so that a folded row equals ra_merge's bit for bit
+// when the output element is fmaf(w_new, o_new, fmaf(w_state, o_state, 0)).
+struct FoldWeights {
+  float L, w_state, w_new;
+};
+__device__ __forceinline__ FoldWeights fold_weights(float lse_state, float lse_new) {
+  float mx = -INFINITY;
+  mx = fmaxf(mx, lse_state);
+  mx = fmaxf(mx, lse_new);
+  const float sh = (mx == -INFINITY) ? 0.f : mx;
+  float tot = 0.f;
+  tot += expf(lse_state - sh);
+  tot += expf(lse_new - sh);
+  const bool empty = !(tot > 0.f);
+  FoldWeights f;
+  f.L = empty ? -INFINITY : sh + logf(tot);
+  f.w_state = empty ? 0.f : expf(lse_state - f.L);
+  f.w_new = empty ? 0.f : expf(lse_new - f.L);
+  return f;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

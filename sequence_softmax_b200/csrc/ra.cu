@@ -203,6 +203,39 @@ ra_status check_dtype_d(ra_dtype dt, int d) {
   return RA_OK;
 }
 
+// ra_partial and ra_partial_fold: one Q block against one KV chunk, the result written as a
+// new partial state (fold == 0) or merged into the caller's (fold == 1).
+ra_status partial_impl(const void* q, const void* k, const void* v, ra_dtype dt, int B, int H, int64_t Lq,
+                       int64_t Lk, int d, float scale, int causal, int64_t q_tok0, int64_t q_tok_stride,
+                       int64_t k_tok0, int64_t k_tok_stride, float* o_partial, float* lse, int fold,
+                       cudaStream_t stream) {
+  if (B < 0 || H < 0 || Lq < 0 || Lk < 0) return RA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return RA_ERR_INVALID_ARG;
+  if (q_tok_stride < 1 || k_tok_stride < 1) return RA_ERR_INVALID_ARG;
+  ra_status st = check_dtype_d(dt, d);
+  if (st != RA_OK) return st;
+  if ((int64_t)B * H > 0x7FFFFFFF) return RA_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || Lq == 0) return RA_OK;
+  if (!q || !o_partial || !lse || !aligned16(q) || !aligned16(o_partial) || !aligned16(lse)) return RA_ERR_INVALID_ARG;
+  if (Lk == 0) {
+    if (fold) return RA_OK;  // nothing to fold in: the state stays as it is
+    const int64_t rows = (int64_t)B * H * Lq;
+    fill_empty_kernel<<<592, 256, 0, stream>>>(o_partial, lse, rows, d);
+    return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+  }
+  if (!k || !v || !aligned16(k) || !aligned16(v)) return RA_ERR_INVALID_ARG;
+  Plan pl{};
+  pl.q = q; pl.k = k; pl.v = v; pl.o = o_partial; pl.lse = lse;
+  pl.BH = B * H; pl.d = d; pl.P = 1; pl.layout = RA_LAYOUT_CONTIGUOUS; pl.causal = causal; pl.out_f32 = 1;
+  pl.fold = fold;
+  pl.q_rows = Lq; pl.k_rows = Lk; pl.q_seg_len = Lq; pl.k_seg_len = Lk;
+  pl.q_tok0 = q_tok0; pl.q_tok_stride = q_tok_stride; pl.k_tok0 = k_tok0; pl.k_tok_stride = k_tok_stride;
+  pl.scale = scale;
+  pl.scale_log2 = scale * 1.4426950408889634f;
+  return launch_attention(pl, dt, 1, stream);
+}
+
 }  // namespace
 }  // namespace ra
 
@@ -252,29 +285,17 @@ ra_status ra_partial(const void* q, const void* k, const void* v, ra_dtype dt, i
                      int64_t Lk, int d, float scale, int causal, int64_t q_tok0, int64_t q_tok_stride,
                      int64_t k_tok0, int64_t k_tok_stride, float* o_partial, float* lse, cudaStream_t stream) {
   NvtxRange nvtx_range("ra_partial");
-  if (B < 0 || H < 0 || Lq < 0 || Lk < 0) return RA_ERR_INVALID_ARG;
-  if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_INVALID_ARG;
-  if (causal != 0 && causal != 1) return RA_ERR_INVALID_ARG;
-  if (q_tok_stride < 1 || k_tok_stride < 1) return RA_ERR_INVALID_ARG;
-  ra_status st = check_dtype_d(dt, d);
-  if (st != RA_OK) return st;
-  if ((int64_t)B * H > 0x7FFFFFFF) return RA_ERR_UNSUPPORTED;
-  if (B == 0 || H == 0 || Lq == 0) return RA_OK;
-  if (!q || !o_partial || !lse || !aligned16(q) || !aligned16(o_partial) || !aligned16(lse)) return RA_ERR_INVALID_ARG;
-  if (Lk == 0) {
-    const int64_t rows = (int64_t)B * H * Lq;
-    fill_empty_kernel<<<592, 256, 0, stream>>>(o_partial, lse, rows, d);
-    return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
-  }
-  if (!k || !v || !aligned16(k) || !aligned16(v)) return RA_ERR_INVALID_ARG;
-  Plan pl{};
-  pl.q = q; pl.k = k; pl.v = v; pl.o = o_partial; pl.lse = lse;
-  pl.BH = B * H; pl.d = d; pl.P = 1; pl.layout = RA_LAYOUT_CONTIGUOUS; pl.causal = causal; pl.out_f32 = 1;
-  pl.q_rows = Lq; pl.k_rows = Lk; pl.q_seg_len = Lq; pl.k_seg_len = Lk;
-  pl.q_tok0 = q_tok0; pl.q_tok_stride = q_tok_stride; pl.k_tok0 = k_tok0; pl.k_tok_stride = k_tok_stride;
-  pl.scale = scale;
-  pl.scale_log2 = scale * 1.4426950408889634f;
-  return launch_attention(pl, dt, 1, stream);
+  return partial_impl(q, k, v, dt, B, H, Lq, Lk, d, scale, causal, q_tok0, q_tok_stride, k_tok0, k_tok_stride,
+                      o_partial, lse, 0, stream);
+}
+
+ra_status ra_partial_fold(const void* q, const void* k, const void* v, ra_dtype dt, int B, int H, int64_t Lq,
+                          int64_t Lk, int d, float scale, int causal, int64_t q_tok0, int64_t q_tok_stride,
+                          int64_t k_tok0, int64_t k_tok_stride, float* o_state, float* lse_state,
+                          cudaStream_t stream) {
+  NvtxRange nvtx_range("ra_partial_fold");
+  return partial_impl(q, k, v, dt, B, H, Lq, Lk, d, scale, causal, q_tok0, q_tok_stride, k_tok0, k_tok_stride,
+                      o_state, lse_state, 1, stream);
 }
 
 ra_status ra_merge(const float* o_parts, const float* lse_parts, int n, int64_t rows, int d, void* o_out,

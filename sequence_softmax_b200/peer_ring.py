@@ -280,7 +280,7 @@ def ring_forward_peer(q_local, k_local, v_local, N: int, layout: str = "contiguo
     Arguments and result as ``ring_dist.ring_forward_dist``: q_local, k_local, v_local
     [B, H, N/W, d] on this rank's GPU hold the tokens of virtual position `rank` in
     increasing token order; returns (O_local in the input dtype, lse_local fp32).
-    ``kernels`` (default: the library binding) provides ``partial`` and ``merge``. ``mode``:
+    ``kernels`` (default: the library binding) provides ``partial_fold``. ``mode``:
     "copy" (the default: each block pulled into a local buffer one step ahead, so it crosses
     NVLink once; see ``_Blocks``) or "direct" (the kernels read the owner's buffer).
     """
@@ -298,9 +298,9 @@ def ring_forward_peer(q_local, k_local, v_local, N: int, layout: str = "contiguo
     q_s = _split_segments(q_local, nseg)
     # segment-major, so that each block segment is a contiguous [B, H, L, d] the kernels read in place
     kv = torch.stack([torch.stack(_split_segments(k_local, nseg)), torch.stack(_split_segments(v_local, nseg))])
-    # per query segment: parts[0] = running state, parts[1] = newest partial
-    state = [(torch.zeros(2, *q.shape, device=dev, dtype=torch.float32),
-              torch.full((2, *q.shape[:3]), float("-inf"), device=dev, dtype=torch.float32)) for q in q_s]
+    # running state (O fp32, lse) per query segment
+    state = [(torch.zeros(*q.shape, device=dev, dtype=torch.float32),
+              torch.full(q.shape[:3], float("-inf"), device=dev, dtype=torch.float32)) for q in q_s]
     peers = share(kv, group)
     try:
         sched = ring_schedule(rank, world)
@@ -312,19 +312,15 @@ def ring_forward_peer(q_local, k_local, v_local, N: int, layout: str = "contiguo
                 for qi, qseg in enumerate(segs):
                     if causal and segment_in_future(qseg, kseg):
                         continue
-                    parts_o, parts_l = state[qi]
-                    kern.partial(q_s[qi], kv_src[0, ki], kv_src[1, ki], causal=causal, scale=scale, q_tok0=qseg[0],
-                                 q_tok_stride=qseg[1], k_tok0=kseg[0], k_tok_stride=kseg[1], out=parts_o[1],
-                                 lse=parts_l[1])
-                    merged_o, merged_l = kern.merge(parts_o, parts_l, out_dtype=torch.float32)
-                    parts_o[0].copy_(merged_o)
-                    parts_l[0].copy_(merged_l)
+                    st_o, st_l = state[qi]
+                    kern.partial_fold(q_s[qi], kv_src[0, ki], kv_src[1, ki], st_o, st_l, causal=causal, scale=scale,
+                                      q_tok0=qseg[0], q_tok_stride=qseg[1], k_tok0=kseg[0], k_tok_stride=kseg[1])
             blocks.done(s)
         _fence(group, kv.is_cuda)  # no rank unmaps or frees a buffer another may still read
     finally:
         peers.close()
-    out = torch.cat([o[0] for o, _ in state], dim=2).to(q_local.dtype)
-    lse = torch.cat([l[0] for _, l in state], dim=2)
+    out = torch.cat([o for o, _ in state], dim=2).to(q_local.dtype)
+    lse = torch.cat([l for _, l in state], dim=2)
     return out, lse
 
 

@@ -9,10 +9,10 @@ listing ``ring_attention_forward``; "Ring Attention" glossary, "How Ring Attenti
 K and V travel as one message (lecture 013 notes: one large message instead of two small
 ones), posted before the step's compute so that the transfer overlaps it.
 
-Every arithmetic step runs in the library's kernels: ``ra_partial`` computes the partial
-state of the local queries against the block held (skipped when the block is wholly in the
-queries' future), and ``ra_merge`` folds it into the running (O, lse) state -- the lse
-associativity of the lecture 013 notes applied step by step. PyTorch provides memory,
+Every arithmetic step runs in the library's kernels: ``ra_partial_fold`` computes the
+partial state of the local queries against the block held (skipped when the block is wholly
+in the queries' future) and folds it into the running (O, lse) state in the same kernel --
+the lse associativity of the lecture 013 notes applied step by step. PyTorch provides memory,
 streams and the process group.
 
 The exchange uses the process group's point-to-point operations: with NCCL on CUDA tensors
@@ -113,7 +113,7 @@ def ring_forward_dist(q_local, k_local, v_local, N: int, layout: str = "contiguo
     holding the tokens of virtual position `rank` in increasing token order (for zig-zag,
     chunk rank followed by chunk 2W-1-rank). Returns (O_local [B, H, N/W, d] in the input
     dtype, lse_local [B, H, N/W] fp32) for the same tokens. ``kernels`` (default: the library
-    binding) provides ``partial`` and ``merge``.
+    binding) provides ``partial_fold``.
     """
     kern = binding if kernels is None else kernels
     world = dist.get_world_size(group)
@@ -124,18 +124,14 @@ def ring_forward_dist(q_local, k_local, v_local, N: int, layout: str = "contiguo
         raise ValueError("local tensors must hold the N/W tokens of this rank's position")
     scale = d ** -0.5 if scale is None else float(scale)
 
-    # Running state per query segment: parts[0] = running O (fp32), parts[1] = newest partial.
+    # Running state (O fp32, lse) per query segment, folded into by every visited block.
     dev = q_local.device
     q_segs, offs = [], 0
     for seg in segs:
         q_segs.append((q_local[:, :, offs:offs + seg[2]].contiguous(), seg, offs))
         offs += seg[2]
-    state = []
-    for qs, seg, _ in q_segs:
-        rows = seg[2]
-        parts_o = torch.zeros(2, B, H, rows, d, device=dev, dtype=torch.float32)
-        parts_l = torch.full((2, B, H, rows), float("-inf"), device=dev, dtype=torch.float32)
-        state.append((parts_o, parts_l))
+    state = [(torch.zeros(B, H, seg[2], d, device=dev, dtype=torch.float32),
+              torch.full((B, H, seg[2]), float("-inf"), device=dev, dtype=torch.float32)) for _, seg, _ in q_segs]
 
     kv = torch.stack([k_local, v_local]).contiguous()     # one K||V message
     kv_next = torch.empty_like(kv)
@@ -148,23 +144,20 @@ def ring_forward_dist(q_local, k_local, v_local, N: int, layout: str = "contiguo
             kk = kv[0][:, :, koff:koff + kseg[2]].contiguous() if len(k_segs) > 1 else kv[0]
             vv = kv[1][:, :, koff:koff + kseg[2]].contiguous() if len(k_segs) > 1 else kv[1]
             koff += kseg[2]
-            for (qs, qseg, _), (parts_o, parts_l) in zip(q_segs, state):
+            for (qs, qseg, _), (st_o, st_l) in zip(q_segs, state):
                 if causal and segment_in_future(qseg, kseg):
                     continue
-                kern.partial(qs, kk, vv, causal=causal, scale=scale, q_tok0=qseg[0], q_tok_stride=qseg[1],
-                             k_tok0=kseg[0], k_tok_stride=kseg[1], out=parts_o[1], lse=parts_l[1])
-                merged_o, merged_l = kern.merge(parts_o, parts_l, out_dtype=torch.float32)
-                parts_o[0].copy_(merged_o)
-                parts_l[0].copy_(merged_l)
+                kern.partial_fold(qs, kk, vv, st_o, st_l, causal=causal, scale=scale, q_tok0=qseg[0],
+                                  q_tok_stride=qseg[1], k_tok0=kseg[0], k_tok_stride=kseg[1])
         if handle is not None:
             kv_next = ex.finish(handle)
             kv, kv_next = kv_next, kv
 
     out = torch.empty_like(q_local)
     lse = torch.empty(B, H, n_local, device=dev, dtype=torch.float32)
-    for (qs, seg, off), (parts_o, parts_l) in zip(q_segs, state):
-        out[:, :, off:off + seg[2]].copy_(parts_o[0])
-        lse[:, :, off:off + seg[2]].copy_(parts_l[0])
+    for (qs, seg, off), (st_o, st_l) in zip(q_segs, state):
+        out[:, :, off:off + seg[2]].copy_(st_o)
+        lse[:, :, off:off + seg[2]].copy_(st_l)
     return out, lse
 
 

@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.ra_abi_version() == 2
+    assert lib.ra_abi_version() == 3
     from sequence_softmax_b200 import binding
     assert binding.ABI_VERSION == lib.ra_abi_version()
     assert binding.load().ra_abi_version() == binding.ABI_VERSION
@@ -105,6 +105,31 @@ def test_partial_rejects(lib, kw, code):
 
 def test_partial_empty_is_noop(lib):
     assert _partial(lib, Lq=0) == binding.RA_OK
+
+
+def _partial_fold(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, dt=1, B=1, H=1, Lq=128, Lk=128, d=64, scale=0.1, causal=0,
+             q_tok0=0, q_ts=1, k_tok0=0, k_ts=1, o=FAKE, lse=FAKE, stream=None)
+    a.update(kw)
+    return lib.ra_partial_fold(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Lq=-1), binding.RA_ERR_INVALID_ARG),
+    (dict(q_ts=0), binding.RA_ERR_INVALID_ARG),
+    (dict(d=32), binding.RA_ERR_UNSUPPORTED),
+    (dict(lse=None), binding.RA_ERR_INVALID_ARG),
+    (dict(o=None), binding.RA_ERR_INVALID_ARG),
+    (dict(causal=2), binding.RA_ERR_INVALID_ARG),
+])
+def test_partial_fold_rejects(lib, kw, code):
+    assert _partial_fold(lib, **kw) == code
+
+
+def test_partial_fold_empty_chunk_leaves_the_state(lib):
+    """Lq == 0 and Lk == 0 launch nothing (the state is never touched: FAKE is not a real pointer)."""
+    assert _partial_fold(lib, Lq=0) == binding.RA_OK
+    assert _partial_fold(lib, Lk=0) == binding.RA_OK
 
 
 def _merge(lib, **kw):

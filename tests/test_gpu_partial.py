@@ -63,3 +63,42 @@ def test_partials_merge_to_full_attention(cuda):
     out, L = binding.merge(torch.stack(parts_o), torch.stack(parts_l), out_dtype=torch.bfloat16)
     o_ref, l_ref = oracle.attention(to_np(q), to_np(k), to_np(v), d ** -0.5, True)
     compare(to_np(out), to_np(L), o_ref, l_ref, "bf16", "partials+merge")
+
+
+FOLD_CASES = [
+    # dtype, B, H, Lq, Lk, d, causal, q_tok0, k_tok0, k_tok_stride
+    ("bf16", 1, 2, 384, 256, 128, True, 0, 128, 1),      # query rows 0-127 see nothing of the chunk
+    ("bf16", 2, 1, 300, 500, 64, False, 0, 0, 1),
+    ("bf16", 1, 1, 256, 256, 128, True, 0, 3, 4),       # strided keys: striped positions
+    ("f32", 1, 2, 70, 90, 32, True, 40, 10, 1),
+]
+
+
+@pytest.mark.parametrize("case", FOLD_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_partial_fold_equals_partial_then_merge(cuda, case):
+    """ra_partial_fold leaves exactly (bit for bit) the state that ra_partial into a scratch
+    state followed by ra_merge of [state, partial] (fp32 output) would: from the empty state,
+    and from a state whose rows include empty ones (lse = -inf) and finite ones."""
+    kind, B, H, Lq, Lk, d, causal, q_tok0, k_tok0, k_ts = case
+    dtype = torch.float32 if kind == "f32" else torch.bfloat16
+    q, k, v = make_qkv(B, H, Lq, d, dtype, seed=Lq + Lk, device="cuda", Nk=Lk)
+    g = torch.Generator(device="cuda").manual_seed(7)
+    starts = [
+        (torch.zeros(B, H, Lq, d, device="cuda"), torch.full((B, H, Lq), float("-inf"), device="cuda")),
+        (torch.randn(B, H, Lq, d, device="cuda", generator=g),
+         torch.where(torch.rand(B, H, Lq, device="cuda", generator=g) < 0.2, float("-inf"),
+                     torch.randn(B, H, Lq, device="cuda", generator=g) + 5.0)),
+    ]
+    kw = dict(causal=causal, q_tok0=q_tok0, k_tok0=k_tok0, k_tok_stride=k_ts)
+    for o0, l0 in starts:
+        o_p, l_p = binding.partial(q, k, v, **kw)
+        want_o, want_l = binding.merge(torch.stack([o0, o_p]), torch.stack([l0, l_p]), out_dtype=torch.float32)
+        st_o, st_l = o0.clone(), l0.clone()
+        binding.partial_fold(q, k, v, st_o, st_l, **kw)
+        assert binding.get_device_error() == binding.RA_OK
+        assert torch.equal(st_o, want_o) and torch.equal(st_l, want_l)
+    # an empty chunk leaves the state untouched
+    st_o, st_l = starts[1][0].clone(), starts[1][1].clone()
+    binding.partial_fold(q, k[:, :, :0].contiguous(), v[:, :, :0].contiguous(), st_o, st_l, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(st_o, starts[1][0]) and torch.equal(st_l, starts[1][1])

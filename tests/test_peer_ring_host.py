@@ -17,7 +17,18 @@ from .test_ring_dist_host import _OracleKernels
 
 
 class _OracleForwardKernels:
-    """Stand-ins for ``partial`` and ``merge`` on CPU tensors (fp64 oracle)."""
+    """Stand-ins for ``partial_fold`` (with ``partial`` and ``merge``) on CPU tensors (fp64 oracle)."""
+
+    @staticmethod
+    def partial_fold(q, k, v, o_state, lse_state, causal=False, scale=None, q_tok0=0, q_tok_stride=1, k_tok0=0,
+                     k_tok_stride=1):
+        import oracle
+        o, l = oracle.partial(q.numpy(), k.numpy(), v.numpy(), scale, causal, q_tok0, q_tok_stride, k_tok0,
+                              k_tok_stride)
+        mo, ml = oracle.merge(np.stack([o_state.numpy(), o]), np.stack([lse_state.numpy(), l]))
+        o_state.copy_(torch.from_numpy(mo))
+        lse_state.copy_(torch.from_numpy(ml))
+        return o_state, lse_state
 
     @staticmethod
     def partial(q, k, v, causal=False, scale=None, q_tok0=0, q_tok_stride=1, k_tok0=0, k_tok_stride=1, out=None,

@@ -17,7 +17,20 @@ from .test_peer_ring_host import _SharedPool
 
 
 class _OracleKernels:
-    """CPU stand-ins for partial / merge / backward_delta / partial_backward (fp64 oracle)."""
+    """CPU stand-ins for partial_fold / partial / merge / backward_delta / partial_backward (fp64 oracle)."""
+
+    @staticmethod
+    def partial_fold(q, k, v, o_state, lse_state, causal=False, scale=None, q_tok0=0, q_tok_stride=1, k_tok0=0,
+                     k_tok_stride=1):
+        import numpy as np
+
+        import oracle
+        o, l = oracle.partial(q.numpy(), k.numpy(), v.numpy(), scale, causal, q_tok0, q_tok_stride, k_tok0,
+                              k_tok_stride)
+        mo, ml = oracle.merge(np.stack([o_state.numpy(), o]), np.stack([lse_state.numpy(), l]))
+        o_state.copy_(torch.from_numpy(mo))
+        lse_state.copy_(torch.from_numpy(ml))
+        return o_state, lse_state
 
     @staticmethod
     def partial(q, k, v, causal=False, scale=None, q_tok0=0, q_tok_stride=1, k_tok0=0, k_tok_stride=1, out=None,
