@@ -14,7 +14,7 @@ How K||V is read (``mode``): "copy" (the default) pulls each step's block one st
 into a local double buffer with one DMA copy (``cudaMemcpyAsync`` on a copy stream), so the
 block crosses NVLink once while the previous step computes, and the kernels' re-reads of
 its tiles (every query tile pair streams the whole block) stay in this GPU's L2 and memory:
-the survey's "receive into local HBM, then local TMA". "direct" hands the kernels the
+the "receive into local memory, then local TMA" plan. "direct" hands the kernels the
 owner's pointers, so their TMA loads fetch every tile over NVLink as the MMA pipeline
 consumes it, re-reads included.
 
