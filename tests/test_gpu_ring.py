@@ -63,22 +63,30 @@ def test_ring_matches_oracle(cuda, case):
 
 
 RAMP_CASES = [
-    # jump (log2 units per 128-key block), N, d, P, layout, causal
-    (10.0, 1024, 128, 1, "contiguous", False),  # the running max moves past the threshold every block
-    (6.0, 1024, 128, 1, "contiguous", True),    # moves by less than the threshold, then past it
-    (10.0, 1024, 64, 1, "contiguous", True),
-    (10.0, 2048, 128, 4, "contiguous", False),  # ring order: a big jump when the walk wraps
-    (10.0, 2048, 128, 4, "zigzag", True),
-    (6.0, 2048, 128, 4, "striped", True),
+    # jump (log2 units per block), block (keys), N, d, P, layout, causal
+    (10.0, 128, 1024, 128, 1, "contiguous", False),  # the running max moves past the threshold every tile
+    (6.0, 128, 1024, 128, 1, "contiguous", True),    # moves by less than the threshold, then past it
+    (10.0, 128, 1024, 64, 1, "contiguous", True),
+    (10.0, 128, 2048, 128, 4, "contiguous", False),  # ring order: a big jump when the walk wraps
+    (10.0, 128, 2048, 128, 4, "zigzag", True),
+    (6.0, 128, 2048, 128, 4, "striped", True),
+    (10.0, 64, 1024, 128, 1, "contiguous", False),   # jumps in both halves of every tile
+    (10.0, 64, 2048, 128, 4, "zigzag", True),
+    (10.0, 64, 1024, 64, 1, "contiguous", True),
+    (80.0, 64, 1024, 128, 1, "contiguous", False),   # a second half far past the running max
+    (80.0, 64, 2048, 128, 4, "zigzag", True),
+    (80.0, 64, 1024, 64, 2, "striped", True),
 ]
 
 
 @pytest.mark.parametrize("case", RAMP_CASES, ids=lambda c: "-".join(map(str, c)))
 def test_running_max_rescale_matches_oracle(cuda, case):
     """Scores that rise block after block (the score ramp of the inputs module) make the
-    forward move its running maximum, and rescale O and l, while it walks the keys."""
-    jump, N, d, P, layout, causal = case
-    q, k, v = ramp_qkv(N, d, jump, seed=N + P, device="cuda")
+    forward move its running maximum, and rescale O and l, while it walks the keys: at tile
+    starts (128-key blocks), in the middle of tiles too (64-key blocks), and by far more than
+    the threshold within a tile's second half (jumps of 80 log2 units)."""
+    jump, block, N, d, P, layout, causal = case
+    q, k, v = ramp_qkv(N, d, jump, seed=N + P, device="cuda", block=block)
     o, lse = binding.ring_forward(q, k, v, P, causal, layout)
     assert binding.get_device_error() == binding.RA_OK
     o_ref, lse_ref = oracle.attention(to_np(q), to_np(k), to_np(v), d ** -0.5, causal)
