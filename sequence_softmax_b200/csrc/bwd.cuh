@@ -220,6 +220,60 @@ __device__ __forceinline__ void bwd_ds_row64(uint32_t taddr, const float (&p)[64
   bwd_ds_regs64<PER_COL>(dr, p, ndscol, ndsrow, scale, ds);
 }
 
+// bwd_exp_row64 for the 32 columns [OFF, OFF + 32) of the thread's 64, loaded from the TMEM
+// columns at taddr + OFF; fills p[OFF .. OFF + 32).
+template <bool PER_COL, int OFF>
+__device__ __forceinline__ void bwd_exp_part32(uint32_t taddr, const float* nl2col, float nl2row, float sl2,
+                                               bool masked, int lo, int hi, float (&p)[64]) {
+  uint32_t sr[32];
+  RA_TMEM_LD32(taddr + OFF, sr);
+  tmem_wait_ld();
+  RA_REG_FENCE32(sr);
+  const uint64_t sl2x2 = f2_pack(sl2, sl2);
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    float4 L = make_float4(nl2row, nl2row, nl2row, nl2row);
+    if (PER_COL) L = *reinterpret_cast<const float4*>(nl2col + OFF + j);
+    float x0, x1, x2, x3;
+    f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), sl2x2, f2_pack(L.x, L.y)), x0, x1);
+    f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3])), sl2x2, f2_pack(L.z, L.w)), x2,
+              x3);
+    p[OFF + j + 0] = ex2_approx(x0);
+    p[OFF + j + 1] = ex2_approx(x1);
+    p[OFF + j + 2] = ex2_approx(x2);
+    p[OFF + j + 3] = ex2_approx(x3);
+  }
+  if (masked) {
+#pragma unroll
+    for (int j = OFF; j < OFF + 32; ++j) p[j] = (j >= lo && j < hi) ? p[j] : 0.f;
+  }
+}
+
+// bwd_ds_row64 for the 32 columns [OFF, OFF + 32): 16 bf16 pairs from the dP columns at
+// taddr + OFF and p[OFF .. OFF + 32).
+template <bool PER_COL, int OFF>
+__device__ __forceinline__ void bwd_ds_part32(uint32_t taddr, const float (&p)[64], const float* ndscol,
+                                              float ndsrow, float scale, uint32_t (&ds)[16]) {
+  uint32_t dr[32];
+  RA_TMEM_LD32(taddr + OFF, dr);
+  tmem_wait_ld();
+  RA_REG_FENCE32(dr);
+  const uint64_t sc2 = f2_pack(scale, scale), z2 = f2_pack(0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    float4 N = make_float4(ndsrow, ndsrow, ndsrow, ndsrow);
+    if (PER_COL) N = *reinterpret_cast<const float4*>(ndscol + OFF + j);
+    const uint64_t t01 = f2_fma(f2_pack(__uint_as_float(dr[j]), __uint_as_float(dr[j + 1])), sc2, f2_pack(N.x, N.y));
+    const uint64_t t23 =
+        f2_fma(f2_pack(__uint_as_float(dr[j + 2]), __uint_as_float(dr[j + 3])), sc2, f2_pack(N.z, N.w));
+    float a, b, c, d;
+    f2_unpack(f2_fma(f2_pack(p[OFF + j], p[OFF + j + 1]), t01, z2), a, b);
+    f2_unpack(f2_fma(f2_pack(p[OFF + j + 2], p[OFF + j + 3]), t23, z2), c, d);
+    ds[j / 2] = pack_bf16x2(a, b);
+    ds[j / 2 + 1] = pack_bf16x2(c, d);
+  }
+}
+
 // ceil(num / den) clamped to [0, cap] for num > 0, den >= 1, with a 32-bit division when the
 // result is below the cap (the per-tile causal bound; 64-bit division is slow on the GPU).
 __device__ __forceinline__ int ceil_div_clamped(int64_t num, int64_t den, int cap) {

@@ -29,7 +29,9 @@
 //                   and -lse_i log2e, -D_i scale (read a tile ahead) into a 2-slot ring
 //   warp 9          MMA issuer (the whole warp loops, one elected lane issues); order per
 //                   tile: dP(i), dV(i), S(i+1), dK(i), so that P(i+1) is computed while
-//                   dK(i) runs
+//                   dK(i) runs. P and dS are released in two halves of 32 queries per
+//                   thread: the k-steps of dV (dK) over the first halves run while the
+//                   second halves are computed (1.4% on the 128K-token causal backward).
 //
 // Tensor memory (512 columns at d = 128): S^T/P^T [0,128) | dP^T/dS^T [128,256) | dV | dK.
 // MMAs issued by one thread execute in order, so S(i+1) overwrites P(i) only after dV(i)
@@ -67,7 +69,7 @@ struct BwCfg {
   static constexpr int DO_OFF = Q_OFF + NQ * TILE_BYTES;
   static constexpr int LD_OFF = DO_OFF + NDO * TILE_BYTES;  // slot s: -lse log2e [128], -D scale [128]
   static constexpr int BAR_OFF = LD_OFF + 2 * 2 * BWD_TILE * 4;
-  static constexpr int NBAR = 1 + 2 * NQ + 2 * NDO + 4 + 6;
+  static constexpr int NBAR = 1 + 2 * NQ + 2 * NDO + 4 + 8;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16;
   static constexpr int COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
@@ -104,7 +106,7 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
   auto bar_ld_empty = [&](int sl) { return bar0 + 8u * (3 + 2 * C::NQ + 2 * C::NDO + sl); };
   const uint32_t bar_s_full = bar0 + 8u * (5 + 2 * C::NQ + 2 * C::NDO), bar_dp_full = bar_s_full + 8u,
                  bar_p_ready = bar_s_full + 16u, bar_ds_ready = bar_s_full + 24u, bar_acc_done = bar_s_full + 32u,
-                 bar_drain = bar_s_full + 40u;
+                 bar_drain = bar_s_full + 40u, bar_p_half = bar_s_full + 48u, bar_ds_half = bar_s_full + 56u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
 
@@ -133,6 +135,8 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     mbar_init(bar_dp_full, 1);
     mbar_init(bar_p_ready, 256);
     mbar_init(bar_ds_ready, 256);
+    mbar_init(bar_p_half, 256);
+    mbar_init(bar_ds_half, 256);
     mbar_init(bar_acc_done, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -284,14 +288,27 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           tc_commit(bar_dp_full);
         }
         __syncwarp();
+        // P^T pairs: queries 0-63 in columns [0, 32), queries 64-127 in [64, 96); each half
+        // of a warpgroup's columns (k-steps 0,1 | 2,3 and 4,5 | 6,7) is released on its own.
+        if (!(ok = wait_all(bar_p_half, pi))) break;
+        tc_fence_after_sync();
+        if (elect_one()) {
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int kk = (h & 1) + (h >> 1) * 4;
+            mma_bf16_ts(tDV, tS + kk * 8 + (kk >= 4 ? 32 : 0), desc(ldo_mn + mnoff(kk)), C::IDESC_KMN,
+                        (i > 0 || h > 0) ? 1u : 0u);
+          }
+        }
+        __syncwarp();
         if (!(ok = wait_all(bar_p_ready, pi))) break;
         tc_fence_after_sync();
         if (elect_one()) {
-          // P^T pairs: queries 0-63 in columns [0, 32), queries 64-127 in [64, 96).
 #pragma unroll
-          for (int kk = 0; kk < BWD_TILE / 16; ++kk)
-            mma_bf16_ts(tDV, tS + kk * 8 + (kk >= 4 ? 32 : 0), desc(ldo_mn + mnoff(kk)), C::IDESC_KMN,
-                        (i > 0 || kk > 0) ? 1u : 0u);
+          for (int h = 0; h < 4; ++h) {
+            const int kk = 2 + (h & 1) + (h >> 1) * 4;
+            mma_bf16_ts(tDV, tS + kk * 8 + (kk >= 4 ? 32 : 0), desc(ldo_mn + mnoff(kk)), C::IDESC_KMN, 1u);
+          }
           tc_commit(bar_do_empty(sd));  // dO(i) is last read by dV(i)
         }
         __syncwarp();
@@ -303,14 +320,25 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
           if (elect_one()) issue_s(sq1);
           __syncwarp();
         }
+        if (!(ok = wait_all(bar_ds_half, pi))) break;
+        tc_fence_after_sync();
+        if (elect_one()) {
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int kk = (h & 1) + (h >> 1) * 4;
+            mma_bf16_ts(tDK, tDP + kk * 8 + (kk >= 4 ? 32 : 0), desc(lq_mn + mnoff(kk)), C::IDESC_KMN,
+                        (i > 0 || h > 0) ? 1u : 0u);
+          }
+        }
+        __syncwarp();
         if (!(ok = wait_all(bar_ds_ready, pi))) break;
         tc_fence_after_sync();
         if (elect_one()) {
-          // dS^T pairs sit in the dP columns like P^T in the S columns.
 #pragma unroll
-          for (int kk = 0; kk < BWD_TILE / 16; ++kk)
-            mma_bf16_ts(tDK, tDP + kk * 8 + (kk >= 4 ? 32 : 0), desc(lq_mn + mnoff(kk)), C::IDESC_KMN,
-                        (i > 0 || kk > 0) ? 1u : 0u);
+          for (int h = 0; h < 4; ++h) {
+            const int kk = 2 + (h & 1) + (h >> 1) * 4;
+            mma_bf16_ts(tDK, tDP + kk * 8 + (kk >= 4 ? 32 : 0), desc(lq_mn + mnoff(kk)), C::IDESC_KMN, 1u);
+          }
           tc_commit(bar_q_empty(sq));  // Q(i) is last read by dK(i)
           if (i == T - 1) tc_commit(bar_acc_done);
         }
@@ -352,26 +380,42 @@ attn_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full, pi, abort_flag)))) return false;
       tc_fence_after_sync();
       float p[64];
-      bwd_exp_row64<true>(tS + c0, l2s, 0.f, pl.scale_log2, masked, lo - c0, 64, p);
+      // Two halves of 32 queries, each released once stored: P pairs of columns c0 .. c0 + 31
+      // land in the S cells c0 .. c0 + 15, already read, those of c0 + 32 .. c0 + 63 in
+      // c0 + 16 .. c0 + 31.
       {
-        uint32_t pk[32];
+        uint32_t pk[16];
+        bwd_exp_part32<true, 0>(tS + c0, l2s, 0.f, pl.scale_log2, masked, lo - c0, 64, p);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) pk[j] = pack_bf16x2(p[2 * j], p[2 * j + 1]);
-        RA_TMEM_ST32(tS + c0, pk);
+        for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(p[2 * j], p[2 * j + 1]);
+        RA_TMEM_ST16(tS + c0, pk);
         tmem_wait_st();
+        tc_fence_before_sync();
+        mbar_arrive(bar_p_half);
+        bwd_exp_part32<true, 32>(tS + c0, l2s, 0.f, pl.scale_log2, masked, lo - c0, 64, p);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(p[32 + 2 * j], p[33 + 2 * j]);
+        RA_TMEM_ST16(tS + c0 + 16, pk);
+        tmem_wait_st();
+        tc_fence_before_sync();
+        mbar_arrive(bar_p_ready);
       }
-      tc_fence_before_sync();
-      mbar_arrive(bar_p_ready);
 
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(bar_dp_full, pi, abort_flag)))) return false;
       tc_fence_after_sync();
-      // dS^T row (this key) x 64 queries: bf16 pairs into the dP columns just read (A of dK).
-      uint32_t dsk[32];
-      bwd_ds_row64<true>(tDP + c0, p, dls, 0.f, pl.scale, dsk);
-      RA_TMEM_ST32(tDP + c0, dsk);
-      tmem_wait_st();
-      tc_fence_before_sync();
-      mbar_arrive(bar_ds_ready);
+      {
+        uint32_t dsk[16];
+        bwd_ds_part32<true, 0>(tDP + c0, p, dls, 0.f, pl.scale, dsk);
+        RA_TMEM_ST16(tDP + c0, dsk);
+        tmem_wait_st();
+        tc_fence_before_sync();
+        mbar_arrive(bar_ds_half);
+        bwd_ds_part32<true, 32>(tDP + c0, p, dls, 0.f, pl.scale, dsk);
+        RA_TMEM_ST16(tDP + c0 + 16, dsk);
+        tmem_wait_st();
+        tc_fence_before_sync();
+        mbar_arrive(bar_ds_ready);
+      }
       mbar_arrive(bar_ld_empty(sl));  // done with this tile's -lse log2e and -D scale
       ++i;
       return true;

@@ -307,6 +307,14 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])                  \
       : "memory")
 
+#define RA_TMEM_ST16(taddr, r)                                                                            \
+  asm volatile(                                                                                           \
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"\
+      "%16};" ::"r"(taddr),                                                                               \
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),  \
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])                   \
+      : "memory")
+
 // Registers written by tcgen05.ld are valid only after tcgen05.wait::ld. The empty asm with
 // "+r" operands ties later uses of the registers to a point after the wait.
 #define RA_REG_FENCE32(r)                                                                                 \
