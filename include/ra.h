@@ -140,6 +140,14 @@ ra_status ra_merge(const float* o_parts, const float* lse_parts, int n, int64_t 
  *
  * Needs N % n_chunks == 0 (N % (2 n_chunks) == 0 for zig-zag) and n_chunks >= 1.
  * N == 0, B == 0 or H == 0 is a no-op.
+ *
+ * Row-max skip (bf16 with lse given, B * H <= 65535): two short kernels first write each
+ * head's largest key norm into every lse slot of the head, using the first rows of o as
+ * scratch; the attention kernel reads its rows' slots before it writes them. A warp then
+ * skips a tile's row max when |q| max|k| scale log2(e) of each of its rows is within 24
+ * log2 units of the running max: no exponential can exceed 2^24, and the result is exact up
+ * to rounding as with the max. Until the call completes on `stream`, o and lse hold these
+ * intermediate values. Keep |V| below 2^72 (fp32 O stays finite with exponentials <= 2^24).
  */
 ra_status ra_ring_forward(const void* q, const void* k, const void* v, ra_dtype dt,
                           int B, int H, int64_t N, int d, float scale, int n_chunks, int causal,

@@ -29,6 +29,10 @@
 // true row max exceeds it by more than RESCALE_LOG2 (in log2 units); until then exp2 values
 // stay <= 2^RESCALE_LOG2 and l and O keep sharing the same stale max, so the result is
 // exact up to rounding.
+//
+// With a key-norm bound (keybound.cuh), a warp also skips the row max of a tile when, for
+// each of its rows, |q| max|k| scale log2(e) <= m + MAXSKIP_LOG2: no score of the tile can then
+// take an exponential above 2^MAXSKIP_LOG2, and m is kept as it is.
 #pragma once
 
 #include "common.cuh"
@@ -44,6 +48,9 @@ constexpr int TC_WARP_PRODUCER = 8;
 constexpr int TC_WARP_MMA = 9;
 constexpr int TC_TMEM_COLS = 512;
 constexpr float RESCALE_LOG2 = 8.0f;
+// Exponentials stay <= 2^MAXSKIP_LOG2 on tiles whose max is skipped: l <= 2^55 for 2^31 keys,
+// and O stays finite in fp32 while |V| < 2^72.
+constexpr float MAXSKIP_LOG2 = 24.0f;
 
 template <int D>
 struct TcCfg {
@@ -424,6 +431,35 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     float l = 0.f;         // running sum of exp2(s * sl2 - m)
     int n = 0;
     bool ok = true;
+    // Upper bound of this row's scaled scores (log2 units): |q| max|k| sl2, rounded up by a
+    // relative 2^-8 and an absolute 2^-8 that cover the fp32 rounding of the norms and of S.
+    // +inf (never skip) without a key bound and for rows past the segment's end.
+    float bq = INFINITY;
+    if (pl.kbound) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_q_full(t), 0, abort_flag));
+      const int64_t mrow = qb.seg.row0 + qb.seg.stride * li;
+      if (ok && row_valid && in_bounds(mrow < pl.q_rows)) {
+        // |q| of this row from the Q tile (the 128B swizzle permutes 16-byte chunks within
+        // the row, which a sum of squares ignores; the rotation by `row` spreads the banks).
+        const uint8_t* qrow = smem + C::Q_OFF + t * C::TILE_BYTES + row * 128;
+        float ss = 0.f;
+#pragma unroll
+        for (int b = 0; b < C::NBOX; ++b)
+#pragma unroll
+          for (int c8 = 0; c8 < 8; ++c8) {
+            const uint4 u = *reinterpret_cast<const uint4*>(qrow + b * C::BOX_BYTES + ((c8 + row) & 7) * 16);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float lo = __uint_as_float(w[i] << 16), hi = __uint_as_float(w[i] & 0xFFFF0000u);
+              ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+            }
+          }
+        const float kmax = pl.lse[(int64_t)bh * pl.q_rows + mrow];
+        bq = fmaf(sqrtf(ss) * kmax * sl2, 1.00390625f, 0.00390625f);
+        if (!(bq >= 0.f)) bq = INFINITY;  // NaN from non-finite inputs: never skip
+      }
+    }
     for (int s = 0; s < pl.P && ok; ++s) {
       int c = qb.p - s;
       if (c < 0) c += pl.P;
@@ -486,7 +522,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           };
           // The online update as the pages state it: the tile's row max first, then the
           // exponentials with the (conditionally) updated running max.
-          update_max(row_max(sr) * sl2);
+          if (!__all_sync(0xffffffffu, bq <= m + MAXSKIP_LOG2)) update_max(row_max(sr) * sl2);
           exp_half(sr, 0, sl2x2, f2_pack(m == -INFINITY ? 0.f : -m, m == -INFINITY ? 0.f : -m), pk, sum2a, sum2b);
           // P of keys 0-63 is complete: the MMA warp may start PV on it while the second half
           // is computed.

@@ -69,6 +69,7 @@ struct Plan {
   int causal;
   int out_f32;       // 1: O written as fp32 (partial states); 0: O in the input dtype
   int fold;          // 1: o / lse hold a running state that the result is merged into
+  int kbound;        // 1: lse holds each row's max key norm of its head (keybound.cuh)
   int64_t q_rows;    // rows per head in the Q / O buffers
   int64_t k_rows;    // rows per head in the K / V buffers
   int64_t q_seg_len; // rows per Q segment

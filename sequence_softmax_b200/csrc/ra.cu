@@ -9,6 +9,7 @@
 #include "common.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
+#include "keybound.cuh"
 #include "merge.cuh"
 #include "bwd.cuh"
 #include "bwd_tc.cuh"
@@ -104,6 +105,22 @@ ra_status launch_tc(const Plan& pl, int S, cudaStream_t stream) {
   if (grid <= 0) return RA_OK;
   if (grid > 0x7FFFFFFFll) return RA_ERR_UNSUPPORTED;
   attn_fwd_tc_kernel<D><<<(unsigned)grid, TC_THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, pl);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
+// The two passes of keybound.cuh: every lse slot of a head gets the head's largest key norm,
+// with O rows as scratch in between. bf16 only (the tensor-core forward reads the bound).
+template <int D>
+ra_status launch_key_bound(const Plan& pl, cudaStream_t stream) {
+  const int C = (int)(pl.k_rows < KB_MAX_CHUNKS ? pl.k_rows : (int64_t)KB_MAX_CHUNKS);
+  if (pl.k_rows != pl.q_rows || C < 1 || pl.BH > 65535) return RA_ERR_UNSUPPORTED;
+  const int64_t o_row_bytes = (int64_t)D * 2;
+  key_norm_chunk_kernel<D><<<dim3((unsigned)C, (unsigned)pl.BH), KB_THREADS, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(pl.k), pl.k_rows, C, pl.o, o_row_bytes);
+  const int64_t gx_need = (pl.q_rows + 4 * KB_THREADS - 1) / (4 * KB_THREADS);
+  const int64_t gx = gx_need < 1024 ? gx_need : 1024;
+  key_norm_spread_kernel<<<dim3((unsigned)gx, (unsigned)pl.BH), KB_THREADS, 0, stream>>>(pl.o, o_row_bytes, pl.q_rows,
+                                                                                          C, pl.lse);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
@@ -354,6 +371,12 @@ ra_status ra_ring_forward(const void* q, const void* k, const void* v, ra_dtype 
   pl.scale = scale;
   pl.scale_log2 = scale * 1.4426950408889634f;
   const int S = layout == RA_LAYOUT_STRIPED ? n_chunks : 1;
+  if (dt == RA_BF16 && lse && (int64_t)B * H <= 65535) {
+    // Key-norm bound for the row-max skip: lse and O are scratch until the forward writes them.
+    st = d == 128 ? launch_key_bound<128>(pl, stream) : launch_key_bound<64>(pl, stream);
+    if (st != RA_OK) return st;
+    pl.kbound = 1;
+  }
   return launch_attention(pl, dt, S, stream);
 }
 

@@ -19,7 +19,9 @@ Recipe:
   coordinate, projected), for one random unit vector u; V is N(0, 1).
   A query's largest score then grows by about ``jump_log2`` (in log2 units, at the default
   scale d^-1/2) from each key block to the next, so an online softmax that visits the
-  blocks in token order sees its running maximum move at every block.
+  blocks in token order sees its running maximum move at every block. ``spread`` (8 by
+  default) scales the orthogonal component; with a small one the keys are nearly parallel
+  to u and |q| max|k| is close to the largest score, so a norm bound on the scores is tight.
 """
 
 from __future__ import annotations
@@ -138,11 +140,11 @@ RAMP_BLOCK = 128  # keys per block of the score ramp
 
 
 def ramp_qkv(N: int, d: int, jump_log2: float, seed: int = 0, dtype=torch.bfloat16, device="cpu",
-             B: int = 1, H: int = 1, block: int = RAMP_BLOCK):
+             B: int = 1, H: int = 1, block: int = RAMP_BLOCK, spread: float = 8.0):
     """Seeded q, k, v [B, H, N, d] whose scores rise by ~jump_log2 per `block`-key block
     (128 by default; 64 puts a jump in the middle of every 128-key tile as well).
 
-    q_i = 4 u + 0.02 n_i, k_j = (floor(j / block) gamma) u + 8 (I - u u^T) n'_j with gamma
+    q_i = 4 u + 0.02 n_i, k_j = (floor(j / block) gamma) u + spread (I - u u^T) n'_j with gamma
     chosen so that 4 gamma d^-1/2 log2(e) = jump_log2; u is a unit vector, n, n' i.i.d.
     N(0, 1). The orthogonal part barely moves the scores (the queries are nearly parallel to
     u) but keeps the keys of one block apart: without it every key of the dominant block is
@@ -157,6 +159,6 @@ def ramp_qkv(N: int, d: int, jump_log2: float, seed: int = 0, dtype=torch.bfloat
     blk = (torch.arange(N, dtype=torch.float64) // block)[:, None]
     q = a * u + 0.02 * torch.randn(B, H, N, d, generator=g, dtype=torch.float64)
     w = torch.randn(B, H, N, d, generator=g, dtype=torch.float64)
-    k = gamma * blk * u + 8.0 * (w - (w @ u)[..., None] * u)
+    k = gamma * blk * u + spread * (w - (w @ u)[..., None] * u)
     v = torch.randn(B, H, N, d, generator=g, dtype=torch.float64)
     return tuple(t.to(dtype).to(device) for t in (q, k, v))

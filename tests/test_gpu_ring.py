@@ -94,6 +94,33 @@ def test_running_max_rescale_matches_oracle(cuda, case):
     compare(to_np(o), to_np(lse), o_ref, lse_ref, "bf16", str(case))
 
 
+SKIP_CASES = [
+    # jump (log2 units per 128-key block), N, d, P, layout, causal
+    (2.5, 1024, 128, 1, "contiguous", False),  # bound within 24 of the first tile's max: m kept
+    (2.5, 1024, 128, 1, "contiguous", True),
+    (2.5, 1024, 64, 1, "contiguous", False),
+    (2.5, 2048, 128, 2, "zigzag", True),       # a rise of 37.5: skipped and computed maxima mixed
+    (2.5, 2048, 128, 1, "contiguous", False),
+]
+
+
+@pytest.mark.parametrize("case", SKIP_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_row_max_skip_matches_oracle(cuda, case):
+    """Keys nearly parallel to the queries (the ramp with a small spread) make the key-norm
+    bound tight: from the second tile on the forward keeps the first tile's max while the
+    scores rise by up to 17.5 log2 units (exponentials up to ~2^17.5), and on the longer
+    ramp it has to take the row max again part of the way."""
+    jump, N, d, P, layout, causal = case
+    q, k, v = ramp_qkv(N, d, jump, seed=N + d, device="cuda", spread=0.05)
+    o, lse = binding.ring_forward(q, k, v, P, causal, layout)
+    assert binding.get_device_error() == binding.RA_OK
+    o_ref, lse_ref = oracle.attention(to_np(q), to_np(k), to_np(v), d ** -0.5, causal)
+    compare(to_np(o), to_np(lse), o_ref, lse_ref, "bf16", str(case))
+    # without lse the forward has no key bound and always takes the row max
+    o2, _ = binding.ring_forward(q, k, v, P, causal, layout, return_lse=False)
+    compare(to_np(o2), None, o_ref, None, "bf16", str(case) + " no lse")
+
+
 def test_layout_invariance_on_gpu(cuda):
     """Contiguous, striped and zig-zag give the same attention (the layout moves work only)."""
     B, H, N, d, P = 1, 4, 4096, 128, 8

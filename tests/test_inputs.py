@@ -35,3 +35,19 @@ def test_ramp_moves_the_running_max_at_every_block():
         if hi is not None:
             assert step.max() < hi, (jump, step.max())
             assert (step[:, 1:] + step[:, :-1]).min() > 8.0
+
+
+def test_tight_ramp_reaches_the_max_skip_regime():
+    """The small-spread ramp of the max-skip GPU tests: for every row the Cauchy-Schwarz bound
+    |q| max|k| d^-1/2 log2(e), rounded up as the forward rounds it, lies within 22 log2 units
+    of the first key block's row max (so the forward keeps that max from the second tile on,
+    under its 24-unit limit), and the last block's row max is more than 8 above the first
+    (so exponentials pass 2^8, where the conditional rescale alone would have moved m)."""
+    for d in (64, 128):
+        q, k, _ = ramp_qkv(1024, d, 2.5, seed=3, spread=0.05)
+        qq, kk = q[0, 0].double().numpy(), k[0, 0].double().numpy()
+        sl2 = d ** -0.5 / np.log(2.0)
+        bound = np.linalg.norm(qq, axis=1) * np.linalg.norm(kk, axis=1).max() * sl2 * (1 + 2.0 ** -8) + 2.0 ** -8
+        bm = _block_maxima_log2(q, k)
+        assert (bound - bm[:, 0]).max() < 22.0
+        assert (bm[:, -1] - bm[:, 0]).min() > 8.0
