@@ -22,7 +22,8 @@
 
 namespace ra {
 
-constexpr int KB_MAX_CHUNKS = 64;  // key chunks per head in pass 1 (at most the head's rows)
+constexpr int KB_MAX_CHUNKS = 1024;  // key chunks per head in pass 1 (at most the head's rows)
+constexpr int KB_TARGET_BLOCKS = 4096;  // pass 1 grid: enough blocks to keep HBM busy
 constexpr int KB_THREADS = 256;
 
 // NaN-propagating maximum: once a NaN is seen the result stays NaN.

@@ -112,7 +112,11 @@ ra_status launch_tc(const Plan& pl, int S, cudaStream_t stream) {
 // with O rows as scratch in between. bf16 only (the tensor-core forward reads the bound).
 template <int D>
 ra_status launch_key_bound(const Plan& pl, cudaStream_t stream) {
-  const int C = (int)(pl.k_rows < KB_MAX_CHUNKS ? pl.k_rows : (int64_t)KB_MAX_CHUNKS);
+  int64_t C64 = (KB_TARGET_BLOCKS + pl.BH - 1) / pl.BH;  // chunks per head
+  if (C64 < 16) C64 = 16;
+  if (C64 > KB_MAX_CHUNKS) C64 = KB_MAX_CHUNKS;
+  if (C64 > pl.k_rows) C64 = pl.k_rows;
+  const int C = (int)C64;
   if (pl.k_rows != pl.q_rows || C < 1 || pl.BH > 65535) return RA_ERR_UNSUPPORTED;
   const int64_t o_row_bytes = (int64_t)D * 2;
   key_norm_chunk_kernel<D><<<dim3((unsigned)C, (unsigned)pl.BH), KB_THREADS, 0, stream>>>(
