@@ -192,6 +192,21 @@ def merge(o_parts, lse_parts, out_dtype=torch.bfloat16, with_lse: bool = True, o
 HOST_PIPELINE_GROUPS = 4
 
 
+def _pipeline_bounds(BH: int, G: int) -> list[int]:
+    """Group boundaries over BH (batch, head) rows for the host pipeline. Only the first
+    group's input copy and the last group's output copy are not hidden behind a kernel, so
+    those two groups get half the weight of the others (8 rows in 4 groups: 1, 3, 3, 1)."""
+    if G <= 2:
+        return [BH * g // G for g in range(G + 1)]
+    w = [0.5] + [1.0] * (G - 2) + [0.5]
+    tot, acc, bounds = sum(w), 0.0, [0]
+    for x in w:
+        acc += x
+        bounds.append(min(BH, max(bounds[-1] + 1, round(BH * acc / tot))))
+    bounds[-1] = BH
+    return bounds
+
+
 def _ring_forward_host(q, k, v, n_chunks, causal, layout, scale, return_lse, out, lse, stream):
     """ring_forward for host tensors: the (batch, head) rows are processed in up to
     HOST_PIPELINE_GROUPS groups, one library call each, so that the copy of group g + 1's
@@ -220,7 +235,7 @@ def _ring_forward_host(q, k, v, n_chunks, causal, layout, scale, return_lse, out
     compute = torch.cuda.current_stream() if stream is None else stream
     h2d, d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     G = max(1, min(HOST_PIPELINE_GROUPS, BH))
-    bounds = [BH * g // G for g in range(G + 1)]
+    bounds = _pipeline_bounds(BH, G)
     for g in range(G):
         a, b = bounds[g], bounds[g + 1]
         if a == b:

@@ -229,3 +229,18 @@ def test_product_path_does_not_reach_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
+
+
+def test_host_pipeline_groups_cover_every_row_once():
+    """The host-buffer forward's head groups: contiguous, non-empty, covering [0, BH), with
+    the first and last groups no larger than the middle ones (their copies are not hidden)."""
+    from sequence_softmax_b200.binding import _pipeline_bounds
+    for BH in range(1, 70):
+        for G in range(1, min(BH, 6) + 1):
+            b = _pipeline_bounds(BH, G)
+            assert b[0] == 0 and b[-1] == BH and len(b) == G + 1
+            sizes = [b[i + 1] - b[i] for i in range(G)]
+            assert all(s >= 1 for s in sizes), (BH, G, b)
+            if G >= 3:
+                assert max(sizes[0], sizes[-1]) <= min(sizes[1:-1]) + 1, (BH, G, sizes)
+    assert _pipeline_bounds(8, 4) == [0, 1, 4, 7, 8]
