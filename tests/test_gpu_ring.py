@@ -121,6 +121,19 @@ def test_row_max_skip_matches_oracle(cuda, case):
     compare(to_np(o2), None, o_ref, None, "bf16", str(case) + " no lse")
 
 
+@pytest.mark.parametrize("scale", [0.05, 0.3, 1.0])
+def test_explicit_scale_matches_oracle(cuda, scale):
+    """A softmax scale other than d^-1/2. At 0.05 the key-norm bound is ~11 log2 units and the
+    row-max skip fires from the second tile; at 0.3 and 1.0 it is far above the scores (and
+    at 1.0 each row's softmax is nearly one-hot), so every tile takes the max."""
+    B, H, N, d, P = 1, 2, 2048, 128, 4
+    q, k, v = make_qkv(B, H, N, d, torch.bfloat16, seed=31, device="cuda")
+    o, lse = binding.ring_forward(q, k, v, P, True, "zigzag", scale=scale)
+    assert binding.get_device_error() == binding.RA_OK
+    o_ref, lse_ref = oracle.attention(to_np(q), to_np(k), to_np(v), scale, True)
+    compare(to_np(o), to_np(lse), o_ref, lse_ref, "bf16", f"scale {scale}")
+
+
 def test_layout_invariance_on_gpu(cuda):
     """Contiguous, striped and zig-zag give the same attention (the layout moves work only)."""
     B, H, N, d, P = 1, 4, 4096, 128, 8
