@@ -511,7 +511,7 @@ class CountingKernels:
         fn = getattr(self._binding, name)
 
         def call(*args, **kwargs):
-            self.launches += 1  # partial_fold: one kernel launch per call
+            self.launches += 1  # partial_fold and key_norm_max: one kernel launch per call
             return fn(*args, **kwargs)
         return call
 
@@ -585,7 +585,8 @@ def run_ring(a, w):
         "roofline": {"bound": "tensor", "achieved": per_gpu, "peak": peak, "unit": "TFLOP/s",
                      "frac": per_gpu / peak, "traffic": None, "peak_source": f"{pk['source']} bf16 burst",
                      "note": "per-GPU step throughput of the ring (ra_partial_fold's attn_fwd_tc_kernel<128> "
-                             "launches and the exchange), not one launch",
+                             "launches, one ra_key_norm_max per folded K segment, and the exchange), "
+                             "not one launch",
                      "kernel": "attn_fwd_tc_kernel<128> via ra_partial_fold"},
         "clocks": clk.summary(),
         "gpu_launches": int(launches.item()),

@@ -97,17 +97,36 @@ ra_status ra_partial(const void* q, const void* k, const void* v, ra_dtype dt,
  *   q, k, v, dt, B, H, Lq, Lk, d, scale, causal, q_tok0 ... k_tok_stride: as ra_partial
  *   o_state    [B, H, Lq, d]  fp32, read and written: the normalised state O
  *   lse_state  [B, H, Lq]     fp32, read and written: the state's lse (-inf: nothing seen yet)
+ *   k_norm_max [B, H]         fp32 or NULL: the largest norm of each head's keys of this
+ *                             chunk, or any larger value (ra_key_norm_max writes it)
  *
- * Afterwards (o_state, lse_state) equal, bit for bit, what ra_partial into a scratch state
- * followed by ra_merge (n = 2, parts [state, new], fp32 output) would leave, without the
- * scratch state, the merge launch or the copies back. Start a ring with o_state = 0 and
+ * With k_norm_max NULL, afterwards (o_state, lse_state) equal, bit for bit, what ra_partial
+ * into a scratch state followed by ra_merge (n = 2, parts [state, new], fp32 output) would
+ * leave, without the scratch state, the merge launch or the copies back. With k_norm_max
+ * (bf16 only; ignored for fp32), a warp skips a tile's row max as ra_ring_forward does, which
+ * changes only the rounding; |V| must then stay below 2^72. A value below a key's true norm
+ * breaks that guarantee: exponentials may then overflow. Start a ring with o_state = 0 and
  * lse_state = -inf. Lq == 0 and Lk == 0 leave the state as it is. The state must not overlap
  * q, k or v.
  */
 ra_status ra_partial_fold(const void* q, const void* k, const void* v, ra_dtype dt,
                           int B, int H, int64_t Lq, int64_t Lk, int d, float scale, int causal,
                           int64_t q_tok0, int64_t q_tok_stride, int64_t k_tok0, int64_t k_tok_stride,
-                          float* o_state, float* lse_state, cudaStream_t stream);
+                          float* o_state, float* lse_state, const float* k_norm_max, cudaStream_t stream);
+
+/*
+ * ra_key_norm_max -- the largest L2 norm of each head's keys, the key half of the bound
+ * |q| max|k| scale log2(e) on a row's scaled scores (Cauchy-Schwarz) that lets the forward
+ * keep its running max on a tile: see ra_ring_forward and ra_partial_fold.
+ *   k           [B, H, Lk, d]  bf16 (d in {64, 128}); read
+ *   k_norm_max  [B, H]         fp32, written: max over j of |k_j|, rounded as fp32 sums of
+ *                              squares and a square root (+inf if a key holds inf or NaN;
+ *                              0 when Lk == 0)
+ * RA_ERR_UNSUPPORTED for fp32 keys or B * H > 65535. The array is first set to zero on
+ * `stream` (a memset, no allocation). The pages have no counterpart: it only feeds the skip.
+ */
+ra_status ra_key_norm_max(const void* k, ra_dtype dt, int B, int H, int64_t Lk, int d, float* k_norm_max,
+                          cudaStream_t stream);
 
 /*
  * ra_merge -- lse-weighted combination of n partial states, from the associativity
@@ -275,7 +294,7 @@ ra_status ra_selftest_wait_timeout(int64_t limit_ns, cudaStream_t stream);
 
 /* ABI version of this header (incremented on any signature change); ra_abi_version()
  * returns the version the library was built with, so a caller can compare the two. */
-#define RA_ABI_VERSION 3
+#define RA_ABI_VERSION 4
 int ra_abi_version(void);
 
 #ifdef __cplusplus

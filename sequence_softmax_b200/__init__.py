@@ -19,9 +19,9 @@ The binding module loads the shared library on first use and raises if it is mis
 ``sequence_softmax_b200.inputs`` (seeded inputs, workload shapes) imports without it.
 """
 
-__all__ = ["partial", "partial_fold", "merge", "ring_forward", "backward_delta", "partial_backward", "ring_backward",
-           "ring_backward_noalloc", "ring_backward_workspace_bytes", "status_string", "get_device_error",
-           "selftest_wait_timeout", "library_path", "RaError"]
+__all__ = ["partial", "partial_fold", "key_norm_max", "merge", "ring_forward", "backward_delta", "partial_backward",
+           "ring_backward", "ring_backward_noalloc", "ring_backward_workspace_bytes", "status_string",
+           "get_device_error", "selftest_wait_timeout", "library_path", "RaError"]
 
 
 def __getattr__(name):

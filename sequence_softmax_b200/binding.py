@@ -20,7 +20,7 @@ library_path = os.environ.get("RA_LIBRARY", os.path.join(_PKG, "libra.so"))
 RA_OK, RA_ERR_INVALID_ARG, RA_ERR_UNSUPPORTED, RA_ERR_CUDA, RA_ERR_TIMEOUT, RA_ERR_DEVICE_BOUNDS = range(6)
 RA_F32, RA_BF16 = 0, 1
 LAYOUTS = {"contiguous": 0, "striped": 1, "zigzag": 2}
-ABI_VERSION = 3  # the ABI these signatures describe (ra_abi_version() of a matching library)
+ABI_VERSION = 4  # the ABI these signatures describe (ra_abi_version() of a matching library)
 
 # name -> (restype, argtypes) of every symbol include/ra.h declares
 _i64, _i32, _f32, _vp = ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_void_p
@@ -28,7 +28,8 @@ SIGNATURES = {
     "ra_partial": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i64, _i64, _i32, _f32, _i32,
                           _i64, _i64, _i64, _i64, _vp, _vp, _vp]),
     "ra_partial_fold": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i64, _i64, _i32, _f32, _i32,
-                               _i64, _i64, _i64, _i64, _vp, _vp, _vp]),
+                               _i64, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "ra_key_norm_max": (_i32, [_vp, _i32, _i32, _i32, _i64, _i32, _vp, _vp]),
     "ra_merge": (_i32, [_vp, _vp, _i32, _i64, _i32, _vp, _i32, _vp, _vp]),
     "ra_ring_forward": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i64, _i32, _f32, _i32, _i32,
                                _i32, _vp, _vp, _vp]),
@@ -142,9 +143,11 @@ def partial(q, k, v, causal: bool = False, scale: float | None = None,
 
 
 def partial_fold(q, k, v, o_state, lse_state, causal: bool = False, scale: float | None = None,
-                 q_tok0: int = 0, q_tok_stride: int = 1, k_tok0: int = 0, k_tok_stride: int = 1, stream=None):
+                 q_tok0: int = 0, q_tok_stride: int = 1, k_tok0: int = 0, k_tok_stride: int = 1,
+                 k_norm_max=None, stream=None):
     """One query block against one KV chunk, merged in place into the running state
-    (o_state fp32 [B,H,Lq,d], lse_state fp32 [B,H,Lq]); returns them."""
+    (o_state fp32 [B,H,Lq,d], lse_state fp32 [B,H,Lq]); returns them. ``k_norm_max``
+    (fp32 [B,H] from ``key_norm_max(k)``, or None) enables the row-max skip."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o_state, "o_state"), (lse_state, "lse_state")):
         _dev(t, n)
     B, H, Lq, d = q.shape
@@ -155,11 +158,30 @@ def partial_fold(q, k, v, o_state, lse_state, causal: bool = False, scale: float
             or lse_state.dtype != torch.float32:
         raise ValueError("the state is o_state fp32 [B, H, Lq, d] and lse_state fp32 [B, H, Lq]")
     scale = d ** -0.5 if scale is None else float(scale)
+    kmax_ptr = None
+    if k_norm_max is not None:
+        _dev(k_norm_max, "k_norm_max")
+        if k_norm_max.shape != (B, H) or k_norm_max.dtype != torch.float32 or not k_norm_max.is_contiguous():
+            raise ValueError("k_norm_max is a contiguous fp32 [B, H] tensor")
+        kmax_ptr = k_norm_max.data_ptr()
     st = load().ra_partial_fold(q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q), B, H, Lq, Lk, d, scale,
                                 int(bool(causal)), q_tok0, q_tok_stride, k_tok0, k_tok_stride,
-                                o_state.data_ptr(), lse_state.data_ptr(), _stream_ptr(stream))
+                                o_state.data_ptr(), lse_state.data_ptr(), kmax_ptr, _stream_ptr(stream))
     _check(st, "ra_partial_fold")
     return o_state, lse_state
+
+
+def key_norm_max(k, out=None, stream=None):
+    """The largest L2 norm of each head's keys: k bf16 [B, H, Lk, d] -> fp32 [B, H]."""
+    _dev(k, "k")
+    B, H, Lk, d = k.shape
+    out = torch.empty(B, H, device=k.device, dtype=torch.float32) if out is None else out
+    _dev(out, "out")
+    if out.shape != (B, H) or out.dtype != torch.float32 or not out.is_contiguous():
+        raise ValueError("out is a contiguous fp32 [B, H] tensor")
+    st = load().ra_key_norm_max(k.data_ptr(), _dtype_code(k), B, H, Lk, d, out.data_ptr(), _stream_ptr(stream))
+    _check(st, "ra_key_norm_max")
+    return out
 
 
 def merge(o_parts, lse_parts, out_dtype=torch.bfloat16, with_lse: bool = True, out=None, lse=None,

@@ -435,7 +435,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // relative 2^-8 and an absolute 2^-8 that cover the fp32 rounding of the norms and of S.
     // +inf (never skip) without a key bound and for rows past the segment's end.
     float bq = INFINITY;
-    if (pl.kbound) {
+    if (pl.kbound || pl.kmax_head) {
       ok = __all_sync(0xffffffffu, mbar_wait(bar_q_full(t), 0, abort_flag));
       const int64_t mrow = qb.seg.row0 + qb.seg.stride * li;
       if (ok && row_valid && in_bounds(mrow < pl.q_rows)) {
@@ -455,7 +455,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
               ss = fmaf(lo, lo, fmaf(hi, hi, ss));
             }
           }
-        const float kmax = pl.lse[(int64_t)bh * pl.q_rows + mrow];
+        const float kmax = pl.kmax_head ? pl.kmax_head[bh] : pl.lse[(int64_t)bh * pl.q_rows + mrow];
         bq = fmaf(sqrtf(ss) * kmax * sl2, 1.00390625f, 0.00390625f);
         if (!(bq >= 0.f)) bq = INFINITY;  // NaN from non-finite inputs: never skip
       }

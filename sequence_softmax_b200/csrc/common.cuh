@@ -70,6 +70,7 @@ struct Plan {
   int out_f32;       // 1: O written as fp32 (partial states); 0: O in the input dtype
   int fold;          // 1: o / lse hold a running state that the result is merged into
   int kbound;        // 1: lse holds each row's max key norm of its head (keybound.cuh)
+  const float* kmax_head;  // or, when not null: the max key norm of each head [BH]
   int64_t q_rows;    // rows per head in the Q / O buffers
   int64_t k_rows;    // rows per head in the K / V buffers
   int64_t q_seg_len; // rows per Q segment

@@ -16,6 +16,11 @@
 //           chunk values.
 // Pass 2 reads O and writes lse only, so its blocks never race with one another. NaN or inf
 // in K propagates into the bound, and the forward then never skips.
+//
+// ra_key_norm_max (key_norm_max_kernel) writes the same per-head maximum into a caller array
+// instead, for ra_partial_fold: every block folds its chunk's maximum in with an integer
+// atomicMax on the float's bits (the order of non-negative floats, +inf and a positive NaN
+// is that of their bit patterns), after a memset of the array to +0.
 #pragma once
 
 #include "common.cuh"
@@ -42,12 +47,13 @@ __device__ __forceinline__ float kb_sq8(uint4 u) {
   return ss;
 }
 
+// The largest squared norm of key rows [c R, min(rows, (c + 1) R)) of head bh (R = ceil(rows / C)),
+// NaN-propagating; valid in thread 0 of the block. Every thread of the block calls it.
 template <int D>
-__global__ void __launch_bounds__(KB_THREADS) key_norm_chunk_kernel(const __nv_bfloat16* __restrict__ k, int64_t rows,
-                                                                    int C, void* o, int64_t o_row_bytes) {
+__device__ __forceinline__ float kb_block_max_sq(const __nv_bfloat16* __restrict__ k, int64_t rows, int C, int c,
+                                                 int bh) {
   constexpr int LPR = D / 8;     // lanes per key row, 16 bytes each
   constexpr int RPW = 32 / LPR;  // key rows per warp step
-  const int c = blockIdx.x, bh = blockIdx.y;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int sub = lane / LPR, part = lane % LPR;
   const int64_t R = (rows + C - 1) / C;
@@ -68,10 +74,30 @@ __global__ void __launch_bounds__(KB_THREADS) key_norm_chunk_kernel(const __nv_b
   __shared__ float s_best[KB_THREADS / 32];
   if (lane == 0) s_best[warp] = best;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    float b = 0.f;
+  float b = 0.f;
+  if (threadIdx.x == 0)
     for (int w = 0; w < KB_THREADS / 32; ++w) b = kb_max(b, s_best[w]);
-    *reinterpret_cast<float*>(static_cast<char*>(o) + ((int64_t)bh * rows + c) * o_row_bytes) = sqrtf(b);
+  return b;
+}
+
+template <int D>
+__global__ void __launch_bounds__(KB_THREADS) key_norm_chunk_kernel(const __nv_bfloat16* __restrict__ k, int64_t rows,
+                                                                    int C, void* o, int64_t o_row_bytes) {
+  const float b = kb_block_max_sq<D>(k, rows, C, blockIdx.x, blockIdx.y);
+  if (threadIdx.x == 0)
+    *reinterpret_cast<float*>(static_cast<char*>(o) + ((int64_t)blockIdx.y * rows + blockIdx.x) * o_row_bytes) =
+        sqrtf(b);
+}
+
+// kmax[bh] = max(kmax[bh], largest key norm of chunk c); kmax starts at +0. A NaN becomes +inf,
+// so that the bound of a head with a non-finite key is +inf whatever the NaN's sign bit.
+template <int D>
+__global__ void __launch_bounds__(KB_THREADS) key_norm_max_kernel(const __nv_bfloat16* __restrict__ k, int64_t rows,
+                                                                  int C, float* __restrict__ kmax) {
+  const float b = kb_block_max_sq<D>(k, rows, C, blockIdx.x, blockIdx.y);
+  if (threadIdx.x == 0) {
+    const float n = (b != b) ? INFINITY : sqrtf(b);
+    atomicMax(reinterpret_cast<int*>(kmax + blockIdx.y), __float_as_int(n));
   }
 }
 

@@ -229,7 +229,7 @@ ra_status check_dtype_d(ra_dtype dt, int d) {
 ra_status partial_impl(const void* q, const void* k, const void* v, ra_dtype dt, int B, int H, int64_t Lq,
                        int64_t Lk, int d, float scale, int causal, int64_t q_tok0, int64_t q_tok_stride,
                        int64_t k_tok0, int64_t k_tok_stride, float* o_partial, float* lse, int fold,
-                       cudaStream_t stream) {
+                       const float* k_norm_max, cudaStream_t stream) {
   if (B < 0 || H < 0 || Lq < 0 || Lk < 0) return RA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return RA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return RA_ERR_INVALID_ARG;
@@ -246,10 +246,12 @@ ra_status partial_impl(const void* q, const void* k, const void* v, ra_dtype dt,
     return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
   }
   if (!k || !v || !aligned16(k) || !aligned16(v)) return RA_ERR_INVALID_ARG;
+  if (k_norm_max && (reinterpret_cast<uintptr_t>(k_norm_max) & 3u)) return RA_ERR_INVALID_ARG;
   Plan pl{};
   pl.q = q; pl.k = k; pl.v = v; pl.o = o_partial; pl.lse = lse;
   pl.BH = B * H; pl.d = d; pl.P = 1; pl.layout = RA_LAYOUT_CONTIGUOUS; pl.causal = causal; pl.out_f32 = 1;
   pl.fold = fold;
+  pl.kmax_head = dt == RA_BF16 ? k_norm_max : nullptr;  // the fp32 kernel always takes the row max
   pl.q_rows = Lq; pl.k_rows = Lk; pl.q_seg_len = Lq; pl.k_seg_len = Lk;
   pl.q_tok0 = q_tok0; pl.q_tok_stride = q_tok_stride; pl.k_tok0 = k_tok0; pl.k_tok_stride = k_tok_stride;
   pl.scale = scale;
@@ -307,16 +309,44 @@ ra_status ra_partial(const void* q, const void* k, const void* v, ra_dtype dt, i
                      int64_t k_tok0, int64_t k_tok_stride, float* o_partial, float* lse, cudaStream_t stream) {
   NvtxRange nvtx_range("ra_partial");
   return partial_impl(q, k, v, dt, B, H, Lq, Lk, d, scale, causal, q_tok0, q_tok_stride, k_tok0, k_tok_stride,
-                      o_partial, lse, 0, stream);
+                      o_partial, lse, 0, nullptr, stream);
 }
 
 ra_status ra_partial_fold(const void* q, const void* k, const void* v, ra_dtype dt, int B, int H, int64_t Lq,
                           int64_t Lk, int d, float scale, int causal, int64_t q_tok0, int64_t q_tok_stride,
                           int64_t k_tok0, int64_t k_tok_stride, float* o_state, float* lse_state,
-                          cudaStream_t stream) {
+                          const float* k_norm_max, cudaStream_t stream) {
   NvtxRange nvtx_range("ra_partial_fold");
   return partial_impl(q, k, v, dt, B, H, Lq, Lk, d, scale, causal, q_tok0, q_tok_stride, k_tok0, k_tok_stride,
-                      o_state, lse_state, 1, stream);
+                      o_state, lse_state, 1, k_norm_max, stream);
+}
+
+ra_status ra_key_norm_max(const void* k, ra_dtype dt, int B, int H, int64_t Lk, int d, float* k_norm_max,
+                          cudaStream_t stream) {
+  NvtxRange nvtx_range("ra_key_norm_max");
+  if (B < 0 || H < 0 || Lk < 0) return RA_ERR_INVALID_ARG;
+  ra_status st = check_dtype_d(dt, d);
+  if (st != RA_OK) return st;
+  if (dt != RA_BF16) return RA_ERR_UNSUPPORTED;
+  const int64_t BH = (int64_t)B * H;
+  if (BH > 65535) return RA_ERR_UNSUPPORTED;
+  if (BH == 0) return RA_OK;
+  if (!k_norm_max || (reinterpret_cast<uintptr_t>(k_norm_max) & 3u)) return RA_ERR_INVALID_ARG;
+  if (Lk > 0 && (!k || !aligned16(k))) return RA_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(k_norm_max, 0, (size_t)BH * sizeof(float), stream) != cudaSuccess) return RA_ERR_CUDA;
+  if (Lk == 0) return RA_OK;
+  int64_t C64 = (KB_TARGET_BLOCKS + BH - 1) / BH;
+  if (C64 < 16) C64 = 16;
+  if (C64 > KB_MAX_CHUNKS) C64 = KB_MAX_CHUNKS;
+  if (C64 > Lk) C64 = Lk;
+  const dim3 grid((unsigned)C64, (unsigned)BH);
+  if (d == 128)
+    key_norm_max_kernel<128><<<grid, KB_THREADS, 0, stream>>>(static_cast<const __nv_bfloat16*>(k), Lk, (int)C64,
+                                                               k_norm_max);
+  else
+    key_norm_max_kernel<64><<<grid, KB_THREADS, 0, stream>>>(static_cast<const __nv_bfloat16*>(k), Lk, (int)C64,
+                                                              k_norm_max);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
 ra_status ra_merge(const float* o_parts, const float* lse_parts, int n, int64_t rows, int d, void* o_out,

@@ -280,7 +280,9 @@ def ring_forward_peer(q_local, k_local, v_local, N: int, layout: str = "contiguo
     Arguments and result as ``ring_dist.ring_forward_dist``: q_local, k_local, v_local
     [B, H, N/W, d] on this rank's GPU hold the tokens of virtual position `rank` in
     increasing token order; returns (O_local in the input dtype, lse_local fp32).
-    ``kernels`` (default: the library binding) provides ``partial_fold``. ``mode``:
+    ``kernels`` (default: the library binding) provides ``partial_fold`` and, for bf16,
+    ``key_norm_max`` (each K segment's largest key norm per head, read where the segment lives,
+    which lets the folding kernel skip row maxima). ``mode``:
     "copy" (the default: each block pulled into a local buffer one step ahead, so it crosses
     NVLink once; see ``_Blocks``) or "direct" (the kernels read the owner's buffer).
     """
@@ -309,12 +311,16 @@ def ring_forward_peer(q_local, k_local, v_local, N: int, layout: str = "contiguo
         for s, src in enumerate(sched):
             kv_src = blocks.get(s)
             for ki, kseg in enumerate(position_segments(layout, N, world, src)):
+                kmax = None
                 for qi, qseg in enumerate(segs):
                     if causal and segment_in_future(qseg, kseg):
                         continue
+                    if kmax is None and kv_src.dtype == torch.bfloat16:
+                        kmax = kern.key_norm_max(kv_src[0, ki])
                     st_o, st_l = state[qi]
                     kern.partial_fold(q_s[qi], kv_src[0, ki], kv_src[1, ki], st_o, st_l, causal=causal, scale=scale,
-                                      q_tok0=qseg[0], q_tok_stride=qseg[1], k_tok0=kseg[0], k_tok_stride=kseg[1])
+                                      q_tok0=qseg[0], q_tok_stride=qseg[1], k_tok0=kseg[0], k_tok_stride=kseg[1],
+                                      k_norm_max=kmax)
             blocks.done(s)
         _fence(group, kv.is_cuda)  # no rank unmaps or frees a buffer another may still read
     finally:

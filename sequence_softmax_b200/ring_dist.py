@@ -113,7 +113,8 @@ def ring_forward_dist(q_local, k_local, v_local, N: int, layout: str = "contiguo
     holding the tokens of virtual position `rank` in increasing token order (for zig-zag,
     chunk rank followed by chunk 2W-1-rank). Returns (O_local [B, H, N/W, d] in the input
     dtype, lse_local [B, H, N/W] fp32) for the same tokens. ``kernels`` (default: the library
-    binding) provides ``partial_fold``.
+    binding) provides ``partial_fold`` and, for bf16, ``key_norm_max``: each received block's
+    largest key norm per head, which lets the folding kernel skip row maxima.
     """
     kern = binding if kernels is None else kernels
     world = dist.get_world_size(group)
@@ -144,11 +145,14 @@ def ring_forward_dist(q_local, k_local, v_local, N: int, layout: str = "contiguo
             kk = kv[0][:, :, koff:koff + kseg[2]].contiguous() if len(k_segs) > 1 else kv[0]
             vv = kv[1][:, :, koff:koff + kseg[2]].contiguous() if len(k_segs) > 1 else kv[1]
             koff += kseg[2]
+            kmax = None  # per segment, as the peer ring takes it: both rings fold identical values
             for (qs, qseg, _), (st_o, st_l) in zip(q_segs, state):
                 if causal and segment_in_future(qseg, kseg):
                     continue
+                if kmax is None and kk.dtype == torch.bfloat16:
+                    kmax = kern.key_norm_max(kk)
                 kern.partial_fold(qs, kk, vv, st_o, st_l, causal=causal, scale=scale, q_tok0=qseg[0],
-                                  q_tok_stride=qseg[1], k_tok0=kseg[0], k_tok_stride=kseg[1])
+                                  q_tok_stride=qseg[1], k_tok0=kseg[0], k_tok_stride=kseg[1], k_norm_max=kmax)
         if handle is not None:
             kv_next = ex.finish(handle)
             kv, kv_next = kv_next, kv

@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.ra_abi_version() == 3
+    assert lib.ra_abi_version() == 4
     from sequence_softmax_b200 import binding
     assert binding.ABI_VERSION == lib.ra_abi_version()
     assert binding.load().ra_abi_version() == binding.ABI_VERSION
@@ -50,6 +50,8 @@ def test_abi_version_and_status_strings(lib):
 
 
 FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every call below fails validation first
+FAKE_2 = ctypes.c_void_p(0x10002)  # 2-byte aligned only
+FAKE_8 = ctypes.c_void_p(0x10008)  # 8-byte aligned only
 
 
 def _ring(lib, **kw):
@@ -109,7 +111,7 @@ def test_partial_empty_is_noop(lib):
 
 def _partial_fold(lib, **kw):
     a = dict(q=FAKE, k=FAKE, v=FAKE, dt=1, B=1, H=1, Lq=128, Lk=128, d=64, scale=0.1, causal=0,
-             q_tok0=0, q_ts=1, k_tok0=0, k_ts=1, o=FAKE, lse=FAKE, stream=None)
+             q_tok0=0, q_ts=1, k_tok0=0, k_ts=1, o=FAKE, lse=FAKE, kmax=None, stream=None)
     a.update(kw)
     return lib.ra_partial_fold(*a.values())
 
@@ -121,6 +123,7 @@ def _partial_fold(lib, **kw):
     (dict(lse=None), binding.RA_ERR_INVALID_ARG),
     (dict(o=None), binding.RA_ERR_INVALID_ARG),
     (dict(causal=2), binding.RA_ERR_INVALID_ARG),
+    (dict(kmax=FAKE_2), binding.RA_ERR_INVALID_ARG),  # a k_norm_max not 4-byte aligned
 ])
 def test_partial_fold_rejects(lib, kw, code):
     assert _partial_fold(lib, **kw) == code
@@ -130,6 +133,31 @@ def test_partial_fold_empty_chunk_leaves_the_state(lib):
     """Lq == 0 and Lk == 0 launch nothing (the state is never touched: FAKE is not a real pointer)."""
     assert _partial_fold(lib, Lq=0) == binding.RA_OK
     assert _partial_fold(lib, Lk=0) == binding.RA_OK
+
+
+def _key_norm_max(lib, **kw):
+    a = dict(k=FAKE, dt=1, B=1, H=2, Lk=128, d=128, out=FAKE, stream=None)
+    a.update(kw)
+    return lib.ra_key_norm_max(*a.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Lk=-1), binding.RA_ERR_INVALID_ARG),
+    (dict(B=-1), binding.RA_ERR_INVALID_ARG),
+    (dict(dt=0), binding.RA_ERR_UNSUPPORTED),  # fp32 keys: the fp32 kernel takes every row max
+    (dict(d=32), binding.RA_ERR_UNSUPPORTED),
+    (dict(B=256, H=256), binding.RA_ERR_UNSUPPORTED),  # B * H > 65535
+    (dict(out=None), binding.RA_ERR_INVALID_ARG),
+    (dict(out=FAKE_2), binding.RA_ERR_INVALID_ARG),
+    (dict(k=None), binding.RA_ERR_INVALID_ARG),
+    (dict(k=FAKE_8), binding.RA_ERR_INVALID_ARG),  # keys not 16-byte aligned
+])
+def test_key_norm_max_rejects(lib, kw, code):
+    assert _key_norm_max(lib, **kw) == code
+
+
+def test_key_norm_max_no_heads_is_noop(lib):
+    assert _key_norm_max(lib, B=0) == binding.RA_OK
 
 
 def _merge(lib, **kw):

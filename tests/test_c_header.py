@@ -27,6 +27,9 @@ int main(void) {
   if (ra_ring_backward_workspace_bytes(RA_BF16, 1, 2, 256, 128) != 2 * 256 * 4) return 5;
   if (ra_ring_backward_noalloc(0, 0, 0, 0, 0, 0, RA_BF16, 64, 64, 1 << 20, 128, 0.1f, 4, 1, RA_LAYOUT_CONTIGUOUS,
                                0, 0, 0, 0) != RA_ERR_UNSUPPORTED) return 6;
+  if (ra_key_norm_max(0, RA_F32, 1, 2, 128, 128, 0, 0) != RA_ERR_UNSUPPORTED) return 7;
+  if (ra_partial_fold(0, 0, 0, RA_BF16, 1, 1, -1, 128, 128, 0.1f, 0, 0, 1, 0, 1, 0, 0, 0, 0) !=
+      RA_ERR_INVALID_ARG) return 8;
   printf("ok\n");
   return 0;
 }

@@ -102,3 +102,53 @@ def test_partial_fold_equals_partial_then_merge(cuda, case):
     binding.partial_fold(q, k[:, :, :0].contiguous(), v[:, :, :0].contiguous(), st_o, st_l, **kw)
     torch.cuda.synchronize()
     assert torch.equal(st_o, starts[1][0]) and torch.equal(st_l, starts[1][1])
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_key_norm_max_matches_the_norms(cuda, d):
+    """ra_key_norm_max against fp64 norms of the same bf16 keys, for one to 70000 keys per
+    head (one to 683 chunks per head): within fp32 rounding of a sum of squares."""
+    for Lk in (1, 100, 4096, 70000):
+        k = make_qkv(2, 3, Lk, d, torch.bfloat16, seed=Lk + d, device="cuda")[1]
+        k[0, 1] *= 4.0                # heads with different maxima (powers of two: exact)
+        k[1, 2, Lk // 2] *= 16.0
+        got = binding.key_norm_max(k).double().cpu()
+        ref = k.double().norm(dim=-1).amax(dim=-1).cpu()
+        assert torch.allclose(got, ref, rtol=1e-5, atol=0.0), (Lk, (got / ref - 1).abs().max())
+
+
+def test_key_norm_max_edge_cases(cuda):
+    """No keys give 0; a key holding inf or NaN gives +inf for its head and no other."""
+    assert torch.equal(binding.key_norm_max(torch.empty(1, 2, 0, 128, dtype=torch.bfloat16, device="cuda")),
+                       torch.zeros(1, 2, device="cuda"))
+    k = make_qkv(1, 3, 512, 128, torch.bfloat16, seed=5, device="cuda")[1]
+    k[0, 1, 7, 3] = float("inf")
+    k[0, 2, 300, 0] = float("nan")
+    got = binding.key_norm_max(k).cpu()
+    assert torch.isfinite(got[0, 0]) and got[0, 1] == float("inf") and got[0, 2] == float("inf")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_partial_fold_with_key_bound_matches_oracle(cuda, causal, d):
+    """Two KV chunks folded into one state with their ra_key_norm_max bounds, on the tight ramp
+    (keys nearly parallel to the queries, scores rising 17.5 log2 units): the folding kernel
+    keeps the first tile's max where the bound allows. Also with no bound, and with one larger
+    than the true norms (still a valid bound)."""
+    from sequence_softmax_b200.inputs import ramp_qkv
+    N = 2048
+    q, k, v = ramp_qkv(N, d, 2.5, seed=9, device="cuda", spread=0.05)
+    o_ref, lse_ref = oracle.attention(to_np(q), to_np(k), to_np(v), d ** -0.5, causal)
+    for mode in ("bound", "none", "loose"):
+        st_o = torch.zeros(1, 1, N, d, device="cuda")
+        st_l = torch.full((1, 1, N), float("-inf"), device="cuda")
+        for c0 in (0, N // 2):
+            kc, vc = k[:, :, c0:c0 + N // 2].contiguous(), v[:, :, c0:c0 + N // 2].contiguous()
+            kmax = None
+            if mode != "none":
+                kmax = binding.key_norm_max(kc)
+                if mode == "loose":
+                    kmax = kmax * 3.0
+            binding.partial_fold(q, kc, vc, st_o, st_l, causal=causal, k_tok0=c0, k_norm_max=kmax)
+        assert binding.get_device_error() == binding.RA_OK
+        compare(to_np(st_o), to_np(st_l), o_ref, lse_ref, "bf16", f"{mode} causal={causal} d={d}")

@@ -21,7 +21,7 @@ class _OracleForwardKernels:
 
     @staticmethod
     def partial_fold(q, k, v, o_state, lse_state, causal=False, scale=None, q_tok0=0, q_tok_stride=1, k_tok0=0,
-                     k_tok_stride=1):
+                     k_tok_stride=1, k_norm_max=None):
         import oracle
         o, l = oracle.partial(q.numpy(), k.numpy(), v.numpy(), scale, causal, q_tok0, q_tok_stride, k_tok0,
                               k_tok_stride)

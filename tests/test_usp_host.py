@@ -21,7 +21,7 @@ class _OracleKernels:
 
     @staticmethod
     def partial_fold(q, k, v, o_state, lse_state, causal=False, scale=None, q_tok0=0, q_tok_stride=1, k_tok0=0,
-                     k_tok_stride=1):
+                     k_tok_stride=1, k_norm_max=None):
         import numpy as np
 
         import oracle
