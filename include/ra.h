@@ -122,7 +122,7 @@ ra_status ra_partial_fold(const void* q, const void* k, const void* v, ra_dtype 
  *   k_norm_max  [B, H]         fp32, written: max over j of |k_j|, rounded as fp32 sums of
  *                              squares and a square root (+inf if a key holds inf or NaN;
  *                              0 when Lk == 0)
- * RA_ERR_UNSUPPORTED for fp32 keys or B * H > 65535. The array is first set to zero on
+ * RA_ERR_UNSUPPORTED for fp32 keys. The array is first set to zero on
  * `stream` (a memset, no allocation). The pages have no counterpart: it only feeds the skip.
  */
 ra_status ra_key_norm_max(const void* k, ra_dtype dt, int B, int H, int64_t Lk, int d, float* k_norm_max,
@@ -160,7 +160,7 @@ ra_status ra_merge(const float* o_parts, const float* lse_parts, int n, int64_t 
  * Needs N % n_chunks == 0 (N % (2 n_chunks) == 0 for zig-zag) and n_chunks >= 1.
  * N == 0, B == 0 or H == 0 is a no-op.
  *
- * Row-max skip (bf16 with lse given, B * H <= 65535): two short kernels first write each
+ * Row-max skip (bf16 with lse given): two short kernels first write each
  * head's largest key norm into every lse slot of the head, using the first rows of o as
  * scratch; the attention kernel reads its rows' slots before it writes them. A warp then
  * skips a tile's row max when |q| max|k| scale log2(e) of each of its rows is within 24

@@ -80,13 +80,14 @@ __device__ __forceinline__ float kb_block_max_sq(const __nv_bfloat16* __restrict
   return b;
 }
 
+// Grids are one-dimensional (any number of heads): block i takes chunk i % C of head i / C.
 template <int D>
 __global__ void __launch_bounds__(KB_THREADS) key_norm_chunk_kernel(const __nv_bfloat16* __restrict__ k, int64_t rows,
                                                                     int C, void* o, int64_t o_row_bytes) {
-  const float b = kb_block_max_sq<D>(k, rows, C, blockIdx.x, blockIdx.y);
+  const int c = (int)(blockIdx.x % (unsigned)C), bh = (int)(blockIdx.x / (unsigned)C);
+  const float b = kb_block_max_sq<D>(k, rows, C, c, bh);
   if (threadIdx.x == 0)
-    *reinterpret_cast<float*>(static_cast<char*>(o) + ((int64_t)blockIdx.y * rows + blockIdx.x) * o_row_bytes) =
-        sqrtf(b);
+    *reinterpret_cast<float*>(static_cast<char*>(o) + ((int64_t)bh * rows + c) * o_row_bytes) = sqrtf(b);
 }
 
 // kmax[bh] = max(kmax[bh], largest key norm of chunk c); kmax starts at +0. A NaN becomes +inf,
@@ -94,16 +95,18 @@ __global__ void __launch_bounds__(KB_THREADS) key_norm_chunk_kernel(const __nv_b
 template <int D>
 __global__ void __launch_bounds__(KB_THREADS) key_norm_max_kernel(const __nv_bfloat16* __restrict__ k, int64_t rows,
                                                                   int C, float* __restrict__ kmax) {
-  const float b = kb_block_max_sq<D>(k, rows, C, blockIdx.x, blockIdx.y);
+  const int c = (int)(blockIdx.x % (unsigned)C), bh = (int)(blockIdx.x / (unsigned)C);
+  const float b = kb_block_max_sq<D>(k, rows, C, c, bh);
   if (threadIdx.x == 0) {
     const float n = (b != b) ? INFINITY : sqrtf(b);
-    atomicMax(reinterpret_cast<int*>(kmax + blockIdx.y), __float_as_int(n));
+    atomicMax(reinterpret_cast<int*>(kmax + bh), __float_as_int(n));
   }
 }
 
+// Block i writes part i % G of head i / G's lse slots.
 __global__ void __launch_bounds__(KB_THREADS) key_norm_spread_kernel(const void* o, int64_t o_row_bytes, int64_t rows,
-                                                                     int C, float* __restrict__ lse) {
-  const int bh = blockIdx.y;
+                                                                     int C, int G, float* __restrict__ lse) {
+  const int bh = (int)(blockIdx.x / (unsigned)G), part = (int)(blockIdx.x % (unsigned)G);
   __shared__ float s_kmax;
   if (threadIdx.x < 32) {
     float b = 0.f;
@@ -116,7 +119,7 @@ __global__ void __launch_bounds__(KB_THREADS) key_norm_spread_kernel(const void*
   __syncthreads();
   const float kmax = s_kmax;
   float* dst = lse + (int64_t)bh * rows;
-  for (int64_t r = (int64_t)blockIdx.x * KB_THREADS + threadIdx.x; r < rows; r += (int64_t)gridDim.x * KB_THREADS)
+  for (int64_t r = (int64_t)part * KB_THREADS + threadIdx.x; r < rows; r += (int64_t)G * KB_THREADS)
     dst[r] = kmax;
 }
 

@@ -108,23 +108,31 @@ ra_status launch_tc(const Plan& pl, int S, cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
+// Chunks per head of the key-norm passes: about KB_TARGET_BLOCKS blocks in all, at least 16
+// per head where the keys allow, and a one-dimensional grid below 2^31 blocks.
+int key_chunks(int64_t BH, int64_t rows) {
+  int64_t C = (KB_TARGET_BLOCKS + BH - 1) / BH;
+  if (C < 16) C = 16;
+  if (C > KB_MAX_CHUNKS) C = KB_MAX_CHUNKS;
+  if (C * BH > 0x7FFFFFFFll) C = 0x7FFFFFFFll / BH;
+  if (C > rows) C = rows;
+  return (int)C;
+}
+
 // The two passes of keybound.cuh: every lse slot of a head gets the head's largest key norm,
 // with O rows as scratch in between. bf16 only (the tensor-core forward reads the bound).
 template <int D>
 ra_status launch_key_bound(const Plan& pl, cudaStream_t stream) {
-  int64_t C64 = (KB_TARGET_BLOCKS + pl.BH - 1) / pl.BH;  // chunks per head
-  if (C64 < 16) C64 = 16;
-  if (C64 > KB_MAX_CHUNKS) C64 = KB_MAX_CHUNKS;
-  if (C64 > pl.k_rows) C64 = pl.k_rows;
-  const int C = (int)C64;
-  if (pl.k_rows != pl.q_rows || C < 1 || pl.BH > 65535) return RA_ERR_UNSUPPORTED;
+  const int C = key_chunks(pl.BH, pl.k_rows);
+  if (pl.k_rows != pl.q_rows || C < 1) return RA_ERR_UNSUPPORTED;
   const int64_t o_row_bytes = (int64_t)D * 2;
-  key_norm_chunk_kernel<D><<<dim3((unsigned)C, (unsigned)pl.BH), KB_THREADS, 0, stream>>>(
+  key_norm_chunk_kernel<D><<<(unsigned)((int64_t)C * pl.BH), KB_THREADS, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(pl.k), pl.k_rows, C, pl.o, o_row_bytes);
-  const int64_t gx_need = (pl.q_rows + 4 * KB_THREADS - 1) / (4 * KB_THREADS);
-  const int64_t gx = gx_need < 1024 ? gx_need : 1024;
-  key_norm_spread_kernel<<<dim3((unsigned)gx, (unsigned)pl.BH), KB_THREADS, 0, stream>>>(pl.o, o_row_bytes, pl.q_rows,
-                                                                                          C, pl.lse);
+  int64_t G = (pl.q_rows + 4 * KB_THREADS - 1) / (4 * KB_THREADS);  // blocks per head in pass 2
+  if (G > 1024) G = 1024;
+  if (G * pl.BH > 0x7FFFFFFFll) G = 0x7FFFFFFFll / pl.BH;
+  key_norm_spread_kernel<<<(unsigned)(G * pl.BH), KB_THREADS, 0, stream>>>(pl.o, o_row_bytes, pl.q_rows, C, (int)G,
+                                                                            pl.lse);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
@@ -329,23 +337,18 @@ ra_status ra_key_norm_max(const void* k, ra_dtype dt, int B, int H, int64_t Lk, 
   if (st != RA_OK) return st;
   if (dt != RA_BF16) return RA_ERR_UNSUPPORTED;
   const int64_t BH = (int64_t)B * H;
-  if (BH > 65535) return RA_ERR_UNSUPPORTED;
+  if (BH > 0x7FFFFFFF) return RA_ERR_UNSUPPORTED;
   if (BH == 0) return RA_OK;
   if (!k_norm_max || (reinterpret_cast<uintptr_t>(k_norm_max) & 3u)) return RA_ERR_INVALID_ARG;
   if (Lk > 0 && (!k || !aligned16(k))) return RA_ERR_INVALID_ARG;
   if (cudaMemsetAsync(k_norm_max, 0, (size_t)BH * sizeof(float), stream) != cudaSuccess) return RA_ERR_CUDA;
   if (Lk == 0) return RA_OK;
-  int64_t C64 = (KB_TARGET_BLOCKS + BH - 1) / BH;
-  if (C64 < 16) C64 = 16;
-  if (C64 > KB_MAX_CHUNKS) C64 = KB_MAX_CHUNKS;
-  if (C64 > Lk) C64 = Lk;
-  const dim3 grid((unsigned)C64, (unsigned)BH);
+  const int C = key_chunks(BH, Lk);
+  const unsigned grid = (unsigned)((int64_t)C * BH);
   if (d == 128)
-    key_norm_max_kernel<128><<<grid, KB_THREADS, 0, stream>>>(static_cast<const __nv_bfloat16*>(k), Lk, (int)C64,
-                                                               k_norm_max);
+    key_norm_max_kernel<128><<<grid, KB_THREADS, 0, stream>>>(static_cast<const __nv_bfloat16*>(k), Lk, C, k_norm_max);
   else
-    key_norm_max_kernel<64><<<grid, KB_THREADS, 0, stream>>>(static_cast<const __nv_bfloat16*>(k), Lk, (int)C64,
-                                                              k_norm_max);
+    key_norm_max_kernel<64><<<grid, KB_THREADS, 0, stream>>>(static_cast<const __nv_bfloat16*>(k), Lk, C, k_norm_max);
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
@@ -405,7 +408,7 @@ ra_status ra_ring_forward(const void* q, const void* k, const void* v, ra_dtype 
   pl.scale = scale;
   pl.scale_log2 = scale * 1.4426950408889634f;
   const int S = layout == RA_LAYOUT_STRIPED ? n_chunks : 1;
-  if (dt == RA_BF16 && lse && (int64_t)B * H <= 65535) {
+  if (dt == RA_BF16 && lse) {
     // Key-norm bound for the row-max skip: lse and O are scratch until the forward writes them.
     st = d == 128 ? launch_key_bound<128>(pl, stream) : launch_key_bound<64>(pl, stream);
     if (st != RA_OK) return st;

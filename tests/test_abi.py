@@ -146,7 +146,7 @@ def _key_norm_max(lib, **kw):
     (dict(B=-1), binding.RA_ERR_INVALID_ARG),
     (dict(dt=0), binding.RA_ERR_UNSUPPORTED),  # fp32 keys: the fp32 kernel takes every row max
     (dict(d=32), binding.RA_ERR_UNSUPPORTED),
-    (dict(B=256, H=256), binding.RA_ERR_UNSUPPORTED),  # B * H > 65535
+    (dict(B=65536, H=65536), binding.RA_ERR_UNSUPPORTED),  # B * H beyond 2^31 - 1
     (dict(out=None), binding.RA_ERR_INVALID_ARG),
     (dict(out=FAKE_2), binding.RA_ERR_INVALID_ARG),
     (dict(k=None), binding.RA_ERR_INVALID_ARG),

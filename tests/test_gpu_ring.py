@@ -219,3 +219,20 @@ def test_workload_sampled_rows(cuda, name):
     o_ref, lse_ref = _oracle_rows_per_head(qs, k, v, rows, w)
     stats = compare(to_np(o[:, :, ridx]), to_np(lse[:, :, ridx]), o_ref, lse_ref, "bf16", name)
     print(name, stats)
+
+
+def test_more_heads_than_a_grid_dimension(cuda):
+    """65540 heads (B * H beyond 65535): the key-bound passes run one-dimensional grids, so the
+    forward keeps its row-max skip and ra_key_norm_max serves any head count. Sampled heads
+    against the oracle, every head's key bound against torch's norms."""
+    B, H, N, d, P = 2, 32770, 256, 64, 2
+    q, k, v = make_qkv(B, H, N, d, torch.bfloat16, seed=41, device="cuda")
+    o, lse = binding.ring_forward(q, k, v, P, True, "zigzag")
+    assert binding.get_device_error() == binding.RA_OK
+    for b, h in ((0, 0), (0, 32769), (1, 0), (1, 16384), (1, 32769)):
+        o_ref, lse_ref = oracle.attention(to_np(q[b:b + 1, h:h + 1]), to_np(k[b:b + 1, h:h + 1]),
+                                          to_np(v[b:b + 1, h:h + 1]), d ** -0.5, True)
+        compare(to_np(o[b:b + 1, h:h + 1]), to_np(lse[b:b + 1, h:h + 1]), o_ref, lse_ref, "bf16", f"head {b},{h}")
+    kmax = binding.key_norm_max(k)
+    ref = k.float().norm(dim=-1).amax(dim=-1)
+    assert torch.allclose(kmax, ref, rtol=1e-5, atol=0.0)
