@@ -158,7 +158,8 @@ ra_status ra_merge(const float* o_parts, const float* lse_parts, int n, int64_t 
  *   lse        [B, H, N]     fp32, written; may be NULL
  *
  * Needs N % n_chunks == 0 (N % (2 n_chunks) == 0 for zig-zag) and n_chunks >= 1.
- * N == 0, B == 0 or H == 0 is a no-op.
+ * N == 0, B == 0 or H == 0 is a no-op. o and lse must not overlap q, k, v or each other
+ * (RA_ERR_INVALID_ARG).
  *
  * Row-max skip (bf16 with lse given): two short kernels first write each
  * head's largest key norm into every lse slot of the head, using the first rows of o as

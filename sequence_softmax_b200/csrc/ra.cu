@@ -77,6 +77,12 @@ bool make_tile_map(CUtensorMap* map, const void* base, int BH, int64_t rows, int
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Whether the byte ranges [a, a + na) and [b, b + nb) share a byte.
+bool overlaps(const void* a, int64_t na, const void* b, int64_t nb) {
+  const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+  return a && b && na > 0 && nb > 0 && pa < pb + (uintptr_t)nb && pb < pa + (uintptr_t)na;
+}
+
 template <int D>
 ra_status launch_tc(const Plan& pl, int S, cudaStream_t stream) {
   using C = TcCfg<D>;
@@ -399,6 +405,14 @@ ra_status ra_ring_forward(const void* q, const void* k, const void* v, ra_dtype 
   if (!q || !k || !v || !o || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return RA_ERR_INVALID_ARG;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return RA_ERR_INVALID_ARG;
+  {
+    // o and lse are written (and serve as scratch before the attention kernel runs): neither
+    // may share memory with an input or with the other.
+    const int64_t nt = (int64_t)B * H * N * d * (dt == RA_F32 ? 4 : 2), nl = (int64_t)B * H * N * 4;
+    for (const void* in : {q, k, v})
+      if (overlaps(o, nt, in, nt) || overlaps(lse, nl, in, nt)) return RA_ERR_INVALID_ARG;
+    if (overlaps(lse, nl, o, nt)) return RA_ERR_INVALID_ARG;
+  }
   Plan pl{};
   pl.q = q; pl.k = k; pl.v = v; pl.o = o; pl.lse = lse;
   pl.BH = B * H; pl.d = d; pl.P = n_chunks; pl.layout = layout; pl.causal = causal; pl.out_f32 = (dt == RA_F32);

@@ -80,6 +80,22 @@ def test_ring_forward_rejects(lib, kw, code):
     assert _ring(lib, **kw) == code
 
 
+Q_, K_, V_ = (ctypes.c_void_p(a) for a in (0x1000000, 0x2000000, 0x3000000))  # 64 KB tensors, 16 MB apart
+
+
+@pytest.mark.parametrize("o,lse", [
+    (ctypes.c_void_p(0x1008000), None),          # o inside q
+    (ctypes.c_void_p(0x2FFFF00), None),          # o runs into k
+    (V_, None),                                  # o is v
+    (ctypes.c_void_p(0x5000000), ctypes.c_void_p(0x3000400)),  # lse inside v
+    (ctypes.c_void_p(0x5000000), ctypes.c_void_p(0x5008000)),  # lse inside o
+])
+def test_ring_forward_rejects_overlapping_outputs(lib, o, lse):
+    """o and lse are written, and hold key-norm values before the attention kernel runs, so
+    neither may share memory with q, k, v or the other."""
+    assert _ring(lib, q=Q_, k=K_, v=V_, o=o, lse=lse) == binding.RA_ERR_INVALID_ARG
+
+
 def test_ring_forward_empty_is_noop(lib):
     assert _ring(lib, N=0) == binding.RA_OK
     assert _ring(lib, B=0) == binding.RA_OK
