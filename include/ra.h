@@ -122,8 +122,9 @@ ra_status ra_partial_fold(const void* q, const void* k, const void* v, ra_dtype 
  *   k_norm_max  [B, H]         fp32, written: max over j of |k_j|, rounded as fp32 sums of
  *                              squares and a square root (+inf if a key holds inf or NaN;
  *                              0 when Lk == 0)
- * RA_ERR_UNSUPPORTED for fp32 keys. The array is first set to zero on
- * `stream` (a memset, no allocation). The pages have no counterpart: it only feeds the skip.
+ * RA_ERR_UNSUPPORTED for fp32 keys; RA_ERR_INVALID_ARG if k_norm_max overlaps k. The array
+ * is first set to zero on `stream` (a memset, no allocation). The pages have no counterpart:
+ * it only feeds the skip.
  */
 ra_status ra_key_norm_max(const void* k, ra_dtype dt, int B, int H, int64_t Lk, int d, float* k_norm_max,
                           cudaStream_t stream);

@@ -347,6 +347,7 @@ ra_status ra_key_norm_max(const void* k, ra_dtype dt, int B, int H, int64_t Lk, 
   if (BH == 0) return RA_OK;
   if (!k_norm_max || (reinterpret_cast<uintptr_t>(k_norm_max) & 3u)) return RA_ERR_INVALID_ARG;
   if (Lk > 0 && (!k || !aligned16(k))) return RA_ERR_INVALID_ARG;
+  if (overlaps(k_norm_max, BH * 4, k, BH * Lk * d * 2)) return RA_ERR_INVALID_ARG;  // the memset would clobber keys
   if (cudaMemsetAsync(k_norm_max, 0, (size_t)BH * sizeof(float), stream) != cudaSuccess) return RA_ERR_CUDA;
   if (Lk == 0) return RA_OK;
   const int C = key_chunks(BH, Lk);

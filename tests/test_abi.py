@@ -167,6 +167,7 @@ def _key_norm_max(lib, **kw):
     (dict(out=FAKE_2), binding.RA_ERR_INVALID_ARG),
     (dict(k=None), binding.RA_ERR_INVALID_ARG),
     (dict(k=FAKE_8), binding.RA_ERR_INVALID_ARG),  # keys not 16-byte aligned
+    (dict(out=ctypes.c_void_p(0x10100)), binding.RA_ERR_INVALID_ARG),  # inside the keys
 ])
 def test_key_norm_max_rejects(lib, kw, code):
     assert _key_norm_max(lib, **kw) == code
